@@ -1,0 +1,514 @@
+#!/usr/bin/env python3
+"""Benchmark of the packed INT-b decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+Workload (the decode GEMV sweep): W 4096x4096 fp32 ~ N(0, 0.02^2) with 0.1%
+outliers x20, quantized per row to b = 6 bits (the headline width; the whole
+sweep b in {4,5,6,7,8,10,12} x M in {1,4,16} is reported beside it), x bf16
+M = 1.  One step is one decode pass over a pool of distinct packed copies of
+the matrix (more than 4x the L2 size, so no step reads from L2), one fused
+dequantize-GEMV launch per copy, captured in a CUDA graph.
+
+value = packed-weight bytes (codes + scales) streamed per second, whole job.
+Everything else on the JSON line (sweep, quantizer, 27B-class MLP matrices,
+tensor-core prefill, mixed-bit recipe pass, e2e through host buffers, the
+oracle's CPU time, SM clocks) is measured in the same run.
+
+Multi-GPU: the decode pass does not shard; each rank runs an independent
+replica and value is the sum over ranks of the work, divided by the slowest
+rank's time ("scaling": "weak").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+HEADLINE_BITS = 6
+DECODE_BITS = [4, 5, 6, 7, 8, 10, 12]
+DECODE_MS = [1, 4, 16]
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+METRIC = "packed b-bit dequant-GEMV GB/s and % HBM peak at M=1; prefill TFLOP/s"
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "mixed_precision_weight_row_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(profile_name, source_files, launches_bytes_scale=1.0):
+    """DRAM bytes per launch from a committed ncu summary, if still current."""
+    p = os.path.join(ROOT, "profiles", profile_name)
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    if d.get("source_hash") != kernel_source_hash(source_files):
+        return None
+    return float(d["dram_bytes_per_launch"]) * launches_bytes_scale
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.uuid],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.15)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), parts[2], parts[3], parts[4:8]))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = sorted(r[0] for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[4]) if v.lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl != "reference":
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# GPU measurements
+# ----------------------------------------------------------------------------
+
+class Pool:
+    """P distinct device copies of one packed matrix (P * bytes > 4 x L2)."""
+
+    def __init__(self, packed, scales, min_bytes):
+        import torch
+
+        per = packed.numel() + scales.numel() * 4
+        self.P = max(2, -(-min_bytes // per))
+        self.packed = [packed.clone() for _ in range(self.P)]
+        self.scales = [scales.clone() for _ in range(self.P)]
+        self.bytes_each = per
+        torch.cuda.synchronize()
+
+
+def graph_of(fn):
+    import torch
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm the launch path before capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(g, steps, warmup, world=1):
+    """Device time (ms) of `steps` replays of g, max over ranks."""
+    import torch
+
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    return max_over_ranks(ms, world)
+
+
+def decode_setup(mpw, W_gpu, b, l2_bytes):
+    packed, scales = mpw.quantize_pack(W_gpu, b)
+    return Pool(packed, scales, 4 * l2_bytes)
+
+
+def measure_decode(mpw, pool, b, M, K, N, steps, warmup, world=1, x=None):
+    import torch
+
+    import workloads as wl
+
+    if x is None:
+        x = wl.gen_x(M, K, wl.DECODE["x_seed"]).cuda()
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        for i in range(pool.P):
+            mpw.qlinear(x, pool.packed[i], pool.scales[i], b, y=y)
+
+    g = graph_of(step)
+    ms = time_graph(g, steps, warmup, world)
+    launches = steps * pool.P
+    us_per_launch = ms * 1e3 / launches
+    alg_bytes = pool.bytes_each + M * K * 2 + M * N * 2
+    out = {
+        "b": b, "M": M, "pool": pool.P, "us_per_launch": us_per_launch,
+        "weight_GBps": pool.bytes_each / (us_per_launch * 1e3),
+        "alg_GBps": alg_bytes / (us_per_launch * 1e3),
+        "ms_total": ms, "launches": launches, "alg_bytes_per_launch": alg_bytes,
+    }
+    del g
+    return out
+
+
+def measure_quantize(mpw, W_gpu, b, steps, warmup, l2_bytes):
+    import torch
+
+    N, K = W_gpu.shape
+    copies = max(2, -(-4 * l2_bytes // (N * K * 4)))
+    Ws = [W_gpu.clone() for _ in range(copies)]
+    rb = mpw.packed_row_bytes(K, b)
+    packed = torch.empty((N, rb), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((N,), dtype=torch.float32, device="cuda")
+
+    def step():
+        for Wc in Ws:
+            mpw.quantize_pack(Wc, b, packed=packed, scales=scales)
+
+    g = graph_of(step)
+    ms = time_graph(g, steps, warmup)
+    per = ms * 1e3 / (steps * copies)
+    alg = N * K * 4 + N * rb + N * 4
+    return {"b": b, "N": N, "K": K, "us_per_launch": per, "alg_GBps": alg / (per * 1e3),
+            "weights_per_s": N * K / (per * 1e-6), "copies": copies}
+
+
+def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup, pool_n):
+    """Same metric through the public call with host buffers: each step copies
+    pool_n packed matrices and x host->device, runs the GEMV on each and reads
+    y back to the host."""
+    import torch
+
+    dp = [torch.empty_like(packed_host, device="cuda") for _ in range(2)]
+    ds = [torch.empty_like(scales_host, device="cuda") for _ in range(2)]
+    dx = torch.empty_like(x_host, device="cuda")
+    dy = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+
+    def step():
+        dx.copy_(x_host, non_blocking=True)
+        for i in range(pool_n):
+            j = i & 1
+            dp[j].copy_(packed_host, non_blocking=True)
+            ds[j].copy_(scales_host, non_blocking=True)
+            mpw.qlinear(dx, dp[j], ds[j], b, y=dy)
+        y_host.copy_(dy, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    wbytes = pool_n * (packed_host.numel() + scales_host.numel() * 4)
+    return {"value": wbytes * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": wbytes + x_host.numel() * 2,
+            "d2h_bytes_per_step": M * N * 2, "ms_per_step": ms / steps}
+
+
+# ----------------------------------------------------------------------------
+# CPU baseline: the oracle, as it stands
+# ----------------------------------------------------------------------------
+
+def cpu_baseline(seconds=10.0, b=HEADLINE_BITS):
+    """The oracle's decode GEMV (unpack + fp64 dequantize-matmul) on a sample
+    of rows of the same workload, repeated for about `seconds`."""
+    import numpy as np
+
+    import oracle
+    import workloads as wl
+
+    c = wl.DECODE
+    rows = 256
+    W = wl.gen_weight(c["N"], c["K"], c["sigma"], c["w_seed"], c["outlier_frac"], c["outlier_scale"])[:rows]
+    x = wl.gen_x(1, c["K"], c["x_seed"]).float().numpy()
+    packed, s = oracle.quantize_pack(W, b)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        q = oracle.unpack(packed, c["K"], b)
+        oracle.qlinear_ref(x, q, s)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    wbytes = n * (packed.size + s.size * 4)
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    return {"value": wbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} of 4096 rows (b={b}, M=1) x {n} repetitions in {dt:.1f} s; "
+                      f"host has {os.cpu_count()} cores, numpy BLAS threads {threads}"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    steps, warmup = args.steps, args.warmup
+    for _ in range(warmup):
+        cpu_baseline(seconds=0.0)
+    t0 = time.perf_counter()
+    samples = []
+    for _ in range(steps):
+        samples.append(cpu_baseline(seconds=min(5.0, max(0.5, 30.0 / max(steps, 1)))))
+    dt = time.perf_counter() - t0
+    v = sum(s["value"] for s in samples) / len(samples)
+    cb = dict(samples[-1])
+    cb["value"] = v
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": warmup, "ms_per_step": dt * 1e3 / max(steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": decode_config(args, pool=None),
+            "cpu_baseline": cb, "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def decode_config(args, pool):
+    return {"workload": "decode GEMV sweep: W 4096x4096 ~N(0,0.02^2) + 0.1% outliers x20, "
+                        f"b={HEADLINE_BITS}, x bf16 M=1",
+            "N": 4096, "K": 4096, "bits": HEADLINE_BITS, "M": 1,
+            "pool_matrices": pool, "l2": "inputs larger than L2: rotating pool of distinct packed "
+                                         "matrices totalling > 4x L2 per step",
+            "parallelism": f"replicas x{args.gpus}"}
+
+
+# ----------------------------------------------------------------------------
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--quick", action="store_true",
+                    help="headline and e2e only (no sweep, extras or CPU baseline)")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import numpy as np
+    import torch
+
+    import mixed_precision_weight_row_b200 as mpw
+    import workloads as wl
+
+    torch.cuda.set_device(local)
+    dev = torch.cuda.current_device()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    uuid = str(getattr(props, "uuid", ""))
+    uuid = ("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else uuid
+    pk = peaks()
+    c = wl.DECODE
+    N, K = c["N"], c["K"]
+    W_np = wl.gen_weight(N, K, c["sigma"], c["w_seed"], c["outlier_frac"], c["outlier_scale"])
+    W = torch.from_numpy(W_np).cuda()
+
+    # ---- headline: b = 6, M = 1 ----
+    pool = decode_setup(mpw, W, HEADLINE_BITS, l2)
+    x1 = wl.gen_x(1, K, c["x_seed"]).cuda()
+    y1 = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        for i in range(pool.P):
+            mpw.qlinear(x1, pool.packed[i], pool.scales[i], HEADLINE_BITS, y=y1)
+
+    g = graph_of(step)
+    with ClockSampler(uuid) as cs:
+        ms = time_graph(g, args.steps, args.warmup, world)
+    clocks = cs.summary()
+    del g
+    launches = args.steps * pool.P
+    ms_per_step = ms / args.steps
+    weight_bytes_per_step = pool.P * pool.bytes_each
+    value = world * weight_bytes_per_step / (ms_per_step * 1e-3) / 1e9
+    us_launch = ms * 1e3 / launches
+    alg_bytes = pool.bytes_each + K * 2 + N * 2
+    achieved = alg_bytes / (us_launch * 1e-6) / 1e9
+
+    extras = {}
+    if rank == 0 and not args.quick:
+        sweep = []
+        for b in DECODE_BITS:
+            p = pool if b == HEADLINE_BITS else decode_setup(mpw, W, b, l2)
+            for M in DECODE_MS:
+                r = measure_decode(mpw, p, b, M, K, N, max(20, args.steps // 4), 3)
+                r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
+                sweep.append({k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()
+                              if k in ("b", "M", "us_per_launch", "weight_GBps", "alg_GBps", "pct_hbm")})
+            if p is not pool:
+                del p
+                torch.cuda.empty_cache()
+        extras["decode_sweep"] = sweep
+        extras["quantize_pack"] = []
+        for b in (4, 6, 8, 12):
+            r = measure_quantize(mpw, W, b, 20, 3, l2)
+            r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
+            extras["quantize_pack"].append({k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()})
+        mlp = []
+        for name, n_, k_ in wl.MLP27B["shapes"][1:]:
+            Wm = wl.gen_weight_torch(n_, k_, wl.MLP27B["sigma"], 17 + n_)
+            for b in wl.MLP27B["bits"]:
+                pm = decode_setup(mpw, Wm, b, l2)
+                for M in wl.MLP27B["Ms"]:
+                    r = measure_decode(mpw, pm, b, M, k_, n_, 20, 3,
+                                       x=wl.gen_x(M, k_, 1).cuda())
+                    mlp.append({"shape": f"{name} {n_}x{k_}", "b": b, "M": M,
+                                "us_per_launch": round(r["us_per_launch"], 3),
+                                "weight_GBps": round(r["weight_GBps"], 1),
+                                "pct_hbm": round(100 * r["alg_GBps"] / pk["hbm_gbs"], 2)})
+                del pm
+                torch.cuda.empty_cache()
+            del Wm
+            torch.cuda.empty_cache()
+        extras["mlp27b"] = mlp
+
+    # ---- e2e: the public call with host buffers ----
+    packed_h = pool.packed[0].cpu().pin_memory()
+    scales_h = pool.scales[0].cpu().pin_memory()
+    x_h = x1.cpu().pin_memory()
+    e2e = measure_e2e(mpw, packed_h, scales_h, x_h, HEADLINE_BITS, 1, N, K,
+                      max(3, min(args.steps, 10)), 3, pool.P)
+    e2e["value"] = world * e2e["value"]
+
+    traffic = profile_traffic("gemv_decode_b6_m1.json", ["gemv.cu"])
+    roof = {"bound": "hbm", "kernel": "gemv_kernel<6,R=4,MT=1>", "achieved": round(achieved, 1),
+            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+            "traffic": traffic, "alg_bytes_per_launch": alg_bytes,
+            "peak_source": pk["source"] + " (copy bandwidth)"}
+
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": decode_config(args, pool.P),
+            "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+            "pct_hbm_peak": round(100 * value / world / pk["hbm_gbs"], 2)}
+    line.update(extras)
+    if rank == 0 and world == 1 and not args.quick:
+        line["cpu_baseline"] = cpu_baseline(seconds=10.0)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

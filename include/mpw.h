@@ -1,0 +1,183 @@
+/*
+ * mpw.h -- packed INT-b weight rows and the fused dequantize-linear layer on
+ * B200 (sm_100a).  C ABI of libmpw.so.
+ *
+ * What it computes (page title, section):
+ *   - Quantization tutorial (aiknowledge.cn, "量化"), "How quantization works":
+ *     symmetric quantization, scale = max|w| / max_int, q = round(w / scale),
+ *     reconstruction q * scale, one scale per output channel.
+ *   - Same page, "Step 1: symmetric quantization": max_int = 2^(b-1) - 1,
+ *     round half to even, a zero channel takes the scale 1 / max_int.
+ *   - DynaQuant (zingnex forum thread), "Step 3: apply the recipe": one bit
+ *     width per weight matrix; "Custom kernel architecture": packed N-bit
+ *     weights are read from memory, expanded in registers to a tensor-core
+ *     format and multiplied; "Status": bit pack / unpack tools.
+ *
+ * Conventions shared by every entry point
+ *   - W is [N, K] row-major: N output features (rows), K input features.
+ *     One fp32 scale per row: s_n = fl32(max_k |w_nk| / Q), Q = 2^(b-1) - 1,
+ *     an IEEE division; a zero row takes s_n = fl32(1 / Q).
+ *   - Codes q = clamp(rint_half_even(fl32(w / s_n)), -Q, Q), IEEE division.
+ *   - Packed format ("canonical"): row n occupies mpw_packed_row_bytes(K, b)
+ *     bytes starting at packed + n * row_bytes.  Code k of the row is stored
+ *     as b-bit two's complement in bits [k*b, k*b + b) of the row read as a
+ *     little-endian integer (LSB-first along K).  The row is padded with zero
+ *     bits to 16 * ceil(K*b / 128) bytes.
+ *   - bits must be in 4..15, N >= 1, K >= 1.
+ *   - Activations x and outputs y are bfloat16, passed as raw uint16_t bit
+ *     patterns, row-major [M, K] and [M, N].
+ *   - All pointers named "device" are device memory owned by the caller; the
+ *     library never allocates, frees or retains caller memory.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream)
+ *     and returns its status synchronously.  On an argument error nothing is
+ *     launched.  No C++ exception crosses this boundary.
+ *   - Alignment: `packed` must be 16-byte aligned.  Everything else needs
+ *     only its natural alignment.
+ */
+#ifndef MPW_H_
+#define MPW_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MPW_API __attribute__((visibility("default")))
+#else
+#define MPW_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* mpw_stream_t; /* a cudaStream_t */
+
+typedef enum mpw_status {
+  MPW_OK = 0,
+  MPW_E_INVALID_ARG = 1,      /* null pointer, non-positive size, bad count */
+  MPW_E_UNSUPPORTED_BITS = 2, /* bits outside 4..15 */
+  MPW_E_MISALIGNED = 3,       /* pointer alignment rule above violated */
+  MPW_E_CUDA = 4,             /* a CUDA runtime call or launch failed */
+  MPW_E_NONFINITE = 5,        /* reserved: reported through the flag word */
+  MPW_E_TIMEOUT = 6           /* a device-side wait gave up (see mpw_device_error) */
+} mpw_status;
+
+/* Static English text for a status code; never NULL. */
+MPW_API const char* mpw_status_str(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+MPW_API int mpw_version(void);
+
+/* Bytes of one packed row: 16 * ceil(K * bits / 128).  Returns 0 if bits is
+ * outside 4..15 or K < 1. */
+MPW_API size_t mpw_packed_row_bytes(int64_t K, int bits);
+
+/*
+ * mpw_quantize_pack -- per-row symmetric quantization and canonical packing.
+ *   W        device, fp32 [N, K] row-major, finite values (precondition).
+ *   packed   device, uint8 [N, mpw_packed_row_bytes(K, bits)], 16-B aligned;
+ *            every byte, padding included, is written.
+ *   scales   device, fp32 [N]; receives s_n.
+ *   nonfinite_flag  device int32 or NULL.  If not NULL and some w is not
+ *            finite, 1 is stored there (the caller clears it beforehand and
+ *            reads it after synchronising); codes of such rows are undefined.
+ * Pages: tutorial "How quantization works", "Step 1"; DynaQuant "Step 3".
+ */
+MPW_API mpw_status mpw_quantize_pack(const float* W, int64_t N, int64_t K, int bits,
+                             uint8_t* packed, float* scales,
+                             int32_t* nonfinite_flag, mpw_stream_t stream);
+
+/*
+ * mpw_unpack -- canonical packed rows back to sign-extended codes.
+ *   packed   device, uint8 [N, row_bytes], 16-B aligned.
+ *   codes    device, int16 [N, K] row-major.
+ * Pages: DynaQuant "Status" (bit pack / unpack tools).
+ */
+MPW_API mpw_status mpw_unpack(const uint8_t* packed, int64_t N, int64_t K, int bits,
+                      int16_t* codes, mpw_stream_t stream);
+
+/*
+ * mpw_dequantize -- reconstruction w_hat = fl32(q * s_n), fp32 [N, K].
+ * Pages: tutorial "How quantization works" (reconstructed = quantized * scale).
+ */
+MPW_API mpw_status mpw_dequantize(const uint8_t* packed, const float* scales,
+                          int64_t N, int64_t K, int bits, float* W_hat,
+                          mpw_stream_t stream);
+
+/*
+ * mpw_qlinear -- fused dequantize-linear y = x @ (q * s)^T.
+ *   x        device, bf16 [M, K] row-major.
+ *   packed, scales  as produced by mpw_quantize_pack for W [N, K].
+ *   y        device, bf16 [M, N] row-major; y[m, n] is
+ *            bf16_rn(s_n * sum_k x[m, k] * q[n, k]) with an fp32 accumulator.
+ *   M >= 1.  M <= 32 runs the decode GEMV kernel (packed rows streamed once,
+ *   unpacked in registers); larger M runs the prefill GEMM on tcgen05 tensor
+ *   cores with the accumulator in tensor memory.  Codes with b <= 9 are fed
+ *   to the tensor cores as exact bf16 values; wider codes are split into
+ *   256*hi + lo, both exact in bf16, so no code is ever rounded.
+ * Pages: DynaQuant "Custom kernel architecture" (packed N-bit -> registers ->
+ * tensor core; 9-15 bit codes on BF16 tensor cores).
+ */
+MPW_API mpw_status mpw_qlinear(const uint16_t* x, const uint8_t* packed,
+                       const float* scales, int bits, int64_t M, int64_t N,
+                       int64_t K, uint16_t* y, mpw_stream_t stream);
+
+/* Kernel choice for mpw_qlinear_path. */
+typedef enum mpw_path {
+  MPW_PATH_AUTO = 0, /* what mpw_qlinear does */
+  MPW_PATH_GEMV = 1, /* decode kernel for any M (re-streams W per 32 rows of x) */
+  MPW_PATH_GEMM = 2  /* tensor-core prefill kernel for any M */
+} mpw_path;
+
+/* mpw_qlinear with an explicit kernel choice; same arguments and results. */
+MPW_API mpw_status mpw_qlinear_path(const uint16_t* x, const uint8_t* packed,
+                            const float* scales, int bits, int64_t M,
+                            int64_t N, int64_t K, uint16_t* y, int path,
+                            mpw_stream_t stream);
+
+/*
+ * One linear of a recipe stack (DynaQuant "Step 3": every matrix carries its
+ * own bit width).  Activations move between caller-owned "slots".
+ *   packed, scales, N, K, bits  the quantized matrix (device pointers).
+ *   in_slot   index of the slot holding x [M, K] (bf16).
+ *   out_slot  index of the slot receiving y [M, N] (bf16).
+ *   norm_input  if nonzero, the linear reads rms(x) instead of x, where
+ *             rms(v) = bf16(v / sqrt(mean(v^2) + 1e-6)) per row, evaluated in
+ *             fp32.  The normalised input is not written back.
+ */
+typedef struct mpw_linear {
+  const uint8_t* packed;
+  const float* scales;
+  int64_t N;
+  int64_t K;
+  int32_t bits;
+  int32_t in_slot;
+  int32_t out_slot;
+  int32_t norm_input;
+} mpw_linear;
+
+/*
+ * mpw_recipe_run -- apply a per-matrix bit-width recipe to a stack of linears:
+ * launches `count` qlinear kernels in order on `stream` (capturable in a CUDA
+ * graph).  slots[i] are device bf16 buffers; each must hold M * (largest N or
+ * K that touches it) elements.  M must be in 1..32 (the decode pass).
+ * A linear whose in_slot equals its out_slot is rejected.
+ */
+MPW_API mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count,
+                          uint16_t* const* slots, int64_t num_slots, int64_t M,
+                          mpw_stream_t stream);
+
+/*
+ * mpw_device_error -- synchronises the current device, returns in *code the
+ * library's device-side error word (0 = none; 1 = a bounded wait inside a
+ * tensor-core kernel gave up) and clears it.  Returns MPW_E_TIMEOUT when the
+ * word was set, MPW_OK otherwise.
+ */
+MPW_API mpw_status mpw_device_error(int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MPW_H_ */

@@ -1,0 +1,225 @@
+"""Packed INT-b weight rows and the fused dequantize-linear layer on B200.
+
+Thin Python binding over ``libmpw.so`` (C ABI declared in ``include/mpw.h``).
+This module only marshals arguments: it checks tensor dtypes, devices and
+shapes, allocates outputs with torch when the caller does not pass them, and
+forwards raw device pointers and the current CUDA stream.  Every step of the
+computation runs in the library's CUDA kernels; there is no CPU fallback, and
+importing the package fails if the library has not been built.
+
+Build: ``python -m mixed_precision_weight_row_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+__all__ = [
+    "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
+    "dequantize", "qlinear", "Linear", "recipe_run", "device_error", "status_str",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmpw.so")
+
+MPW_OK = 0
+MPW_E_INVALID_ARG = 1
+MPW_E_UNSUPPORTED_BITS = 2
+MPW_E_MISALIGNED = 3
+MPW_E_CUDA = 4
+MPW_E_NONFINITE = 5
+MPW_E_TIMEOUT = 6
+
+PATHS = {"auto": 0, "gemv": 1, "gemm": 2}
+
+
+class MPWError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)} (status {status})")
+
+
+class _Linear(ctypes.Structure):
+    _fields_ = [
+        ("packed", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+        ("N", ctypes.c_int64),
+        ("K", ctypes.c_int64),
+        ("bits", ctypes.c_int32),
+        ("in_slot", ctypes.c_int32),
+        ("out_slot", ctypes.c_int32),
+        ("norm_input", ctypes.c_int32),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m mixed_precision_weight_row_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+    L.mpw_status_str.argtypes = [c_int]
+    L.mpw_status_str.restype = ctypes.c_char_p
+    L.mpw_version.argtypes = []
+    L.mpw_version.restype = c_int
+    L.mpw_packed_row_bytes.argtypes = [i64, c_int]
+    L.mpw_packed_row_bytes.restype = ctypes.c_size_t
+    L.mpw_quantize_pack.argtypes = [vp, i64, i64, c_int, vp, vp, vp, vp]
+    L.mpw_quantize_pack.restype = c_int
+    L.mpw_unpack.argtypes = [vp, i64, i64, c_int, vp, vp]
+    L.mpw_unpack.restype = c_int
+    L.mpw_dequantize.argtypes = [vp, vp, i64, i64, c_int, vp, vp]
+    L.mpw_dequantize.restype = c_int
+    L.mpw_qlinear.argtypes = [vp, vp, vp, c_int, i64, i64, i64, vp, vp]
+    L.mpw_qlinear.restype = c_int
+    L.mpw_qlinear_path.argtypes = [vp, vp, vp, c_int, i64, i64, i64, vp, c_int, vp]
+    L.mpw_qlinear_path.restype = c_int
+    L.mpw_recipe_run.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp]
+    L.mpw_recipe_run.restype = c_int
+    L.mpw_device_error.argtypes = [ctypes.POINTER(i32)]
+    L.mpw_device_error.restype = c_int
+    return L
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.mpw_status_str(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != MPW_OK:
+        raise MPWError(status, where)
+
+
+def _stream(stream=None) -> int:
+    import torch
+
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _need(t, dtype, name, ndim=None):
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+
+
+def packed_row_bytes(K: int, bits: int) -> int:
+    """16 * ceil(K * bits / 128); 0 if bits is outside 4..15 or K < 1."""
+    return int(lib.mpw_packed_row_bytes(int(K), int(bits)))
+
+
+def quantize_pack(W, bits: int, packed=None, scales=None, nonfinite_flag=None, stream=None):
+    """W fp32 [N, K] (CUDA) -> (packed uint8 [N, row_bytes], scales fp32 [N])."""
+    import torch
+
+    _need(W, torch.float32, "W", 2)
+    N, K = W.shape
+    rb = packed_row_bytes(K, bits)
+    if packed is None:
+        packed = torch.empty((N, max(rb, 16)), dtype=torch.uint8, device=W.device)
+    if scales is None:
+        scales = torch.empty((N,), dtype=torch.float32, device=W.device)
+    _need(packed, torch.uint8, "packed")
+    _need(scales, torch.float32, "scales")
+    flag = 0 if nonfinite_flag is None else nonfinite_flag.data_ptr()
+    _check(lib.mpw_quantize_pack(W.data_ptr(), N, K, int(bits), packed.data_ptr(), scales.data_ptr(),
+                                 flag, _stream(stream)), "mpw_quantize_pack")
+    return packed, scales
+
+
+def unpack(packed, K: int, bits: int, codes=None, stream=None):
+    """packed uint8 [N, row_bytes] -> codes int16 [N, K]."""
+    import torch
+
+    _need(packed, torch.uint8, "packed", 2)
+    N = packed.shape[0]
+    if codes is None:
+        codes = torch.empty((N, K), dtype=torch.int16, device=packed.device)
+    _need(codes, torch.int16, "codes")
+    _check(lib.mpw_unpack(packed.data_ptr(), N, int(K), int(bits), codes.data_ptr(), _stream(stream)),
+           "mpw_unpack")
+    return codes
+
+
+def dequantize(packed, scales, K: int, bits: int, out=None, stream=None):
+    """(packed, scales) -> fl32(q * s) as fp32 [N, K]."""
+    import torch
+
+    _need(packed, torch.uint8, "packed", 2)
+    _need(scales, torch.float32, "scales", 1)
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.float32, device=packed.device)
+    _need(out, torch.float32, "out")
+    _check(lib.mpw_dequantize(packed.data_ptr(), scales.data_ptr(), N, int(K), int(bits), out.data_ptr(),
+                              _stream(stream)), "mpw_dequantize")
+    return out
+
+
+def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", stream=None):
+    """y = x @ (q * s)^T with x bf16 [M, K]; returns y bf16 [M, N]."""
+    import torch
+
+    _need(x, torch.bfloat16, "x", 2)
+    _need(packed, torch.uint8, "packed", 2)
+    _need(scales, torch.float32, "scales", 1)
+    M, K = x.shape
+    N = packed.shape[0]
+    if scales.shape[0] != N:
+        raise ValueError("scales must have one entry per packed row")
+    if packed.shape[1] < packed_row_bytes(K, bits):
+        raise ValueError("packed rows are shorter than packed_row_bytes(K, bits)")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(y, torch.bfloat16, "y")
+    _check(lib.mpw_qlinear_path(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits), M, N, K,
+                                y.data_ptr(), PATHS[path], _stream(stream)), "mpw_qlinear")
+    return y
+
+
+@dataclass
+class Linear:
+    """One quantized linear of a recipe stack (see mpw_linear in mpw.h)."""
+    packed: object
+    scales: object
+    N: int
+    K: int
+    bits: int
+    in_slot: int
+    out_slot: int
+    norm_input: bool = False
+
+
+def recipe_run(layers, slots, M: int, stream=None):
+    """Launch every linear of ``layers`` in order (one kernel each)."""
+    arr = (_Linear * len(layers))()
+    for i, L in enumerate(layers):
+        arr[i] = _Linear(L.packed.data_ptr(), L.scales.data_ptr(), int(L.N), int(L.K), int(L.bits),
+                         int(L.in_slot), int(L.out_slot), int(bool(L.norm_input)))
+    ptrs = (ctypes.c_void_p * len(slots))(*[s.data_ptr() for s in slots])
+    _check(lib.mpw_recipe_run(arr, len(layers), ptrs, len(slots), int(M), _stream(stream)),
+           "mpw_recipe_run")
+
+
+def device_error() -> int:
+    """Synchronise; return and clear the library's device-side error word."""
+    code = ctypes.c_int32(0)
+    st = lib.mpw_device_error(ctypes.byref(code))
+    if st not in (MPW_OK, MPW_E_TIMEOUT):
+        _check(st, "mpw_device_error")
+    return int(code.value)

@@ -1,0 +1,197 @@
+// C ABI of libmpw.so: argument validation and kernel dispatch.  See mpw.h for
+// the contract of every entry point.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "mpw.h"
+#include "mpw_internal.h"
+
+namespace mpw {
+
+// Device-side error word: set by bounded waits that give up.
+__device__ int32_t g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_info[kMaxDevices];
+std::mutex g_mutex;
+
+struct AttrEntry {
+  const void* kernel;
+  int device;
+  size_t bytes;
+};
+AttrEntry g_attrs[1024];
+int g_num_attrs = 0;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+mpw_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MPW_OK : MPW_E_CUDA; }
+
+bool bits_ok(int bits) { return bits >= kMinBits && bits <= kMaxBits; }
+
+}  // namespace
+
+const DeviceInfo& device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = 0;
+  DeviceInfo& d = g_info[dev];
+  if (d.device != dev) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (d.device != dev) {
+      int sms = 0, smem = 0;
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+      d.num_sms = sms > 0 ? sms : 1;
+      d.max_smem_optin = smem;
+      d.device = dev;
+    }
+  }
+  return d;
+}
+
+cudaError_t ensure_smem_attr(const void* kernel, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  for (int i = 0; i < g_num_attrs; ++i)
+    if (g_attrs[i].kernel == kernel && g_attrs[i].device == dev && g_attrs[i].bytes >= bytes)
+      return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e != cudaSuccess) return e;
+  if (g_num_attrs < 1024) g_attrs[g_num_attrs++] = AttrEntry{kernel, dev, bytes};
+  return cudaSuccess;
+}
+
+int32_t* device_error_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<int32_t*>(p);
+}
+
+}  // namespace mpw
+
+using namespace mpw;
+
+extern "C" {
+
+const char* mpw_status_str(int status) {
+  switch (status) {
+    case MPW_OK: return "ok";
+    case MPW_E_INVALID_ARG: return "invalid argument";
+    case MPW_E_UNSUPPORTED_BITS: return "bit width outside 4..15";
+    case MPW_E_MISALIGNED: return "misaligned pointer";
+    case MPW_E_CUDA: return "CUDA error";
+    case MPW_E_NONFINITE: return "non-finite input";
+    case MPW_E_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int mpw_version(void) { return 100; }
+
+size_t mpw_packed_row_bytes(int64_t K, int bits) {
+  if (!bits_ok(bits) || K < 1) return 0;
+  return static_cast<size_t>(16 * ((K * bits + 127) / 128));
+}
+
+mpw_status mpw_quantize_pack(const float* W, int64_t N, int64_t K, int bits, uint8_t* packed,
+                             float* scales, int32_t* nonfinite_flag, mpw_stream_t stream) {
+  if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
+  if (W == nullptr || packed == nullptr || scales == nullptr || N < 1 || K < 1) return MPW_E_INVALID_ARG;
+  if (N > 0x7fffffff || K > 0x3fffffff) return MPW_E_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(W, 4) || !aligned(scales, 4) ||
+      (nonfinite_flag != nullptr && !aligned(nonfinite_flag, 4)))
+    return MPW_E_MISALIGNED;
+  return from_cuda(launch_quantize_pack(W, N, K, bits, packed, scales, nonfinite_flag,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mpw_status mpw_unpack(const uint8_t* packed, int64_t N, int64_t K, int bits, int16_t* codes,
+                      mpw_stream_t stream) {
+  if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
+  if (packed == nullptr || codes == nullptr || N < 1 || K < 1) return MPW_E_INVALID_ARG;
+  if (K > 0x3fffffff) return MPW_E_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(codes, 2)) return MPW_E_MISALIGNED;
+  return from_cuda(launch_unpack(packed, N, K, bits, codes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mpw_status mpw_dequantize(const uint8_t* packed, const float* scales, int64_t N, int64_t K, int bits,
+                          float* W_hat, mpw_stream_t stream) {
+  if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
+  if (packed == nullptr || scales == nullptr || W_hat == nullptr || N < 1 || K < 1)
+    return MPW_E_INVALID_ARG;
+  if (K > 0x3fffffff) return MPW_E_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(scales, 4) || !aligned(W_hat, 4)) return MPW_E_MISALIGNED;
+  return from_cuda(
+      launch_dequantize(packed, scales, N, K, bits, W_hat, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mpw_status mpw_qlinear_path(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                            int64_t M, int64_t N, int64_t K, uint16_t* y, int path,
+                            mpw_stream_t stream) {
+  if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
+  if (x == nullptr || packed == nullptr || scales == nullptr || y == nullptr || M < 1 || N < 1 ||
+      K < 1)
+    return MPW_E_INVALID_ARG;
+  if (N > 0x7fffffff || K > 0x3fffffff || M > 0x7fffffff) return MPW_E_INVALID_ARG;
+  if (path < MPW_PATH_AUTO || path > MPW_PATH_GEMM) return MPW_E_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(x, 2) || !aligned(y, 2) || !aligned(scales, 4))
+    return MPW_E_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool want_gemm = path == MPW_PATH_GEMM || (path == MPW_PATH_AUTO && M > 32);
+  if (want_gemm && gemm_supported(M, N, K) && aligned(x, 16)) {
+    return from_cuda(launch_gemm(x, packed, scales, bits, M, N, K, y, device_error_word(), s));
+  }
+  if (path == MPW_PATH_GEMM) return MPW_E_INVALID_ARG;  // shape the GEMM does not take
+  return from_cuda(launch_gemv(x, packed, scales, bits, M, N, K, y, false, s));
+}
+
+mpw_status mpw_qlinear(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                       int64_t M, int64_t N, int64_t K, uint16_t* y, mpw_stream_t stream) {
+  return mpw_qlinear_path(x, packed, scales, bits, M, N, K, y, MPW_PATH_AUTO, stream);
+}
+
+mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count, uint16_t* const* slots,
+                          int64_t num_slots, int64_t M, mpw_stream_t stream) {
+  if (layers == nullptr || slots == nullptr || count < 1 || num_slots < 1 || M < 1 || M > 32)
+    return MPW_E_INVALID_ARG;
+  for (int64_t i = 0; i < count; ++i) {
+    const mpw_linear& L = layers[i];
+    if (!bits_ok(L.bits)) return MPW_E_UNSUPPORTED_BITS;
+    if (L.packed == nullptr || L.scales == nullptr || L.N < 1 || L.K < 1 || L.N > 0x7fffffff ||
+        L.K > 0x3fffffff)
+      return MPW_E_INVALID_ARG;
+    if (L.in_slot < 0 || L.in_slot >= num_slots || L.out_slot < 0 || L.out_slot >= num_slots ||
+        L.in_slot == L.out_slot)
+      return MPW_E_INVALID_ARG;
+    if (slots[L.in_slot] == nullptr || slots[L.out_slot] == nullptr) return MPW_E_INVALID_ARG;
+    if (!aligned(L.packed, 16) || !aligned(L.scales, 4)) return MPW_E_MISALIGNED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (int64_t i = 0; i < count; ++i) {
+    const mpw_linear& L = layers[i];
+    cudaError_t e = launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, M, L.N, L.K,
+                                slots[L.out_slot], L.norm_input != 0, s);
+    if (e != cudaSuccess) return MPW_E_CUDA;
+  }
+  return MPW_OK;
+}
+
+mpw_status mpw_device_error(int32_t* code) {
+  if (code == nullptr) return MPW_E_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MPW_E_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return MPW_E_CUDA;
+  const int32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return MPW_E_CUDA;
+  *code = v;
+  return v != 0 ? MPW_E_TIMEOUT : MPW_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,262 @@
+// Decode GEMV: y[m, n] = bf16(s_n * sum_k x[m, k] * q[n, k]) for a few tokens.
+//
+// DynaQuant, "Custom kernel architecture": the packed N-bit weights are read
+// from memory once, expanded in registers and multiplied; in decode the
+// saving in bytes is the speedup because the layer is bandwidth-bound
+// (quantization tutorial, closing note: decode is memory-bound).
+//
+// Work layout.  A warp owns R consecutive weight rows at a time.  Lane l walks
+// the row in groups of 32 codes (g = l, l+32, ...); one group of one row is
+// exactly B 32-bit words of the packed stream, so the warp reads 128*B
+// contiguous bytes per row per step.  Codes are expanded with one funnel
+// shift and one LOP3 each: the b-bit two's-complement field, with its sign
+// bit flipped, is OR-ed into the mantissa of 2^23, and one FADD removes the
+// 2^23 + 2^(b-1) offset, which gives the code as an exact fp32 integer.
+// x lives in shared memory as fp32, transposed so that lane l's eight float4
+// loads for its group are conflict-free and shared by the R rows.  Partial sums
+// use four accumulators per (row, token) and a final warp reduction; the row
+// scale is applied once, after the sum.
+//
+// CTAs are persistent (grid = min(tasks, resident CTAs)); x is staged once per
+// CTA when it fits in shared memory, else per K-chunk.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mpw_internal.h"
+
+namespace mpw {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr size_t kXSmemBudget = 150 * 1024;
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t v) {
+  return __uint_as_float(static_cast<uint32_t>(v) << 16);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Code j (0..31) of a group held in w[0..B-1] as an exact fp32 integer.
+template <int B>
+__device__ __forceinline__ float code_f32(const uint32_t (&w)[B + 1], int j) {
+  const int o = j * B;
+  const int i = o >> 5, r = o & 31;
+  uint32_t t;
+  if (r == 0) t = w[i];
+  else if (r + B <= 32) t = w[i] >> r;
+  else t = __funnelshift_r(w[i], w[i + 1], r);
+  constexpr uint32_t kMask = (1u << B) - 1u;
+  constexpr uint32_t kMagic = 0x4B000000u | (1u << (B - 1));  // 2^23, sign bit flip
+  constexpr float kOffset = 8388608.0f + static_cast<float>(1 << (B - 1));
+  return __uint_as_float((t & kMask) ^ kMagic) - kOffset;
+}
+
+// Float index of element (group gl, j) of one token in the transposed x tile.
+__device__ __forceinline__ int xs_index(int gl, int j) {
+  return (((gl >> 5) * 8 + (j >> 2)) * 32 + (gl & 31)) * 4 + (j & 3);
+}
+
+// Stage tokens [0, MT) of x, groups [gb, gb + gc) into xs (zeros past K / mt).
+template <int MT, bool NORM>
+__device__ __forceinline__ void stage_x(float* xs, const uint16_t* __restrict__ x, int ldx, int mt,
+                                        int K, int gb, int gc, const float* inv_rms) {
+  const int elems = gc * 32;
+  for (int t = 0; t < MT; ++t) {
+    float* dst = xs + t * elems;
+    const uint16_t* src = x + static_cast<size_t>(t) * ldx;
+    for (int idx = threadIdx.x; idx < elems; idx += kThreads) {
+      const int k = gb * 32 + idx;
+      float v = 0.0f;
+      if (t < mt && k < K) {
+        v = bf16_bits_to_float(__ldg(src + k));
+        if (NORM) v = __bfloat162float(__float2bfloat16_rn(v * inv_rms[t]));
+      }
+      dst[xs_index(idx >> 5, idx & 31)] = v;
+    }
+  }
+}
+
+// 1 / sqrt(mean(x^2) + 1e-6) per token, fp32, fixed reduction order (every
+// CTA computes the same value bit for bit).
+template <int MT>
+__device__ void token_inv_rms(const uint16_t* __restrict__ x, int ldx, int mt, int K, float* out,
+                              float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int t = 0; t < MT; ++t) {
+    float ss = 0.0f;
+    if (t < mt)
+      for (int k = threadIdx.x; k < K; k += kThreads) {
+        const float v = bf16_bits_to_float(__ldg(x + static_cast<size_t>(t) * ldx + k));
+        ss = fmaf(v, v, ss);
+      }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float tot = 0.0f;
+      for (int w = 0; w < kWarps; ++w) tot += red[w];
+      out[t] = 1.0f / sqrtf(tot / static_cast<float>(K) + 1e-6f);
+    }
+    __syncthreads();
+  }
+}
+
+template <int B, int R, int MT, bool NORM>
+__global__ void __launch_bounds__(kThreads)
+gemv_kernel(const uint16_t* __restrict__ x, int mt, const uint8_t* __restrict__ packed,
+            const float* __restrict__ scales, int N, int K, int rw, uint16_t* __restrict__ y,
+            int gc, int num_tasks) {
+  extern __shared__ __align__(16) float xs[];
+  __shared__ float inv_rms[MT];
+  __shared__ float red[kWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = (K + 31) >> 5;
+  const int nchunks = (G + gc - 1) / gc;
+  const uint32_t* pw = reinterpret_cast<const uint32_t*>(packed);
+
+  if (NORM) token_inv_rms<MT>(x, K, mt, K, inv_rms, red);
+
+  for (int task = blockIdx.x; task < num_tasks; task += gridDim.x) {
+    const int row0 = (task * kWarps + warp) * R;
+    float acc[R][MT][4];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int t = 0; t < MT; ++t)
+#pragma unroll
+        for (int a = 0; a < 4; ++a) acc[r][t][a] = 0.0f;
+
+    for (int c = 0; c < nchunks; ++c) {
+      const int gb = c * gc;
+      const int ge = min(G, gb + gc);
+      if (nchunks > 1 || task == static_cast<int>(blockIdx.x)) {
+        __syncthreads();
+        stage_x<MT, NORM>(xs, x, K, mt, K, gb, gc, inv_rms);
+        __syncthreads();
+      }
+      for (int g = gb + lane; g < ge; g += 32) {
+        const int gl = g - gb;
+        uint32_t w[R][B + 1];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const int n = row0 + r;
+          const uint32_t* rowp = pw + static_cast<size_t>(n) * rw + static_cast<size_t>(g) * B;
+          const bool full = n < N && (g + 1) * B <= rw;
+#pragma unroll
+          for (int i = 0; i < B; ++i)
+            w[r][i] = full ? __ldg(rowp + i) : ((n < N && g * B + i < rw) ? __ldg(rowp + i) : 0u);
+          w[r][B] = 0u;
+        }
+        float xv[MT][32];
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          const float4* x4 = reinterpret_cast<const float4*>(xs + t * gc * 32);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const float4 v = x4[((gl >> 5) * 8 + jj) * 32 + (gl & 31)];
+            xv[t][4 * jj + 0] = v.x;
+            xv[t][4 * jj + 1] = v.y;
+            xv[t][4 * jj + 2] = v.z;
+            xv[t][4 * jj + 3] = v.w;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const float q = code_f32<B>(w[r], j);
+#pragma unroll
+            for (int t = 0; t < MT; ++t) acc[r][t][j & 3] = fmaf(xv[t][j], q, acc[r][t][j & 3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int n = row0 + r;
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        float v = (acc[r][t][0] + acc[r][t][1]) + (acc[r][t][2] + acc[r][t][3]);
+        v = warp_sum(v);
+        if (lane == 0 && n < N && t < mt) {
+          const float outv = v * __ldg(scales + n);
+          y[static_cast<size_t>(t) * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(outv));
+        }
+      }
+    }
+  }
+}
+
+template <int B, int R, int MT, bool NORM>
+cudaError_t run_gemv(const uint16_t* x, int mt, const uint8_t* packed, const float* scales, int N,
+                     int K, uint16_t* y, cudaStream_t stream) {
+  const int rw = static_cast<int>(row_words(K, B));
+  const int G = (K + 31) / 32;
+  const int g_round = (G + 31) / 32 * 32;
+  int gc = static_cast<int>(kXSmemBudget / (static_cast<size_t>(MT) * 32 * 4)) / 32 * 32;
+  if (gc > g_round) gc = g_round;
+  const size_t smem = static_cast<size_t>(MT) * gc * 32 * 4;
+  auto kern = gemv_kernel<B, R, MT, NORM>;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kXSmemBudget);
+  if (e != cudaSuccess) return e;
+  const int rows_per_task = kWarps * R;
+  const int num_tasks = (N + rows_per_task - 1) / rows_per_task;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const int resident = per_sm * device_info().num_sms;
+  const int grid = num_tasks < resident ? num_tasks : resident;
+  kern<<<grid, kThreads, smem, stream>>>(x, mt, packed, scales, N, K, rw, y, gc, num_tasks);
+  return cudaGetLastError();
+}
+
+template <int B>
+cudaError_t gemv_bits(const uint16_t* x, int64_t M, const uint8_t* packed, const float* scales,
+                      int64_t N, int64_t K, uint16_t* y, bool norm, cudaStream_t stream) {
+  // passes over the tokens: 2 at a time, a last single one if M is odd
+  for (int64_t m0 = 0; m0 < M; m0 += 2) {
+    const int mt = static_cast<int>(M - m0 >= 2 ? 2 : 1);
+    const uint16_t* xp = x + m0 * K;
+    uint16_t* yp = y + m0 * N;
+    cudaError_t e;
+    if (mt == 2)
+      e = norm ? run_gemv<B, 2, 2, true>(xp, mt, packed, scales, static_cast<int>(N), static_cast<int>(K), yp, stream)
+               : run_gemv<B, 2, 2, false>(xp, mt, packed, scales, static_cast<int>(N), static_cast<int>(K), yp, stream);
+    else
+      e = norm ? run_gemv<B, 4, 1, true>(xp, mt, packed, scales, static_cast<int>(N), static_cast<int>(K), yp, stream)
+               : run_gemv<B, 4, 1, false>(xp, mt, packed, scales, static_cast<int>(N), static_cast<int>(K), yp, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                        int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm_input,
+                        cudaStream_t stream) {
+  switch (bits) {
+    case 4: return gemv_bits<4>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 5: return gemv_bits<5>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 6: return gemv_bits<6>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 7: return gemv_bits<7>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 8: return gemv_bits<8>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 9: return gemv_bits<9>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 10: return gemv_bits<10>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 11: return gemv_bits<11>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 12: return gemv_bits<12>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 13: return gemv_bits<13>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 14: return gemv_bits<14>(x, M, packed, scales, N, K, y, norm_input, stream);
+    case 15: return gemv_bits<15>(x, M, packed, scales, N, K, y, norm_input, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace mpw

@@ -1,0 +1,150 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before launching anything.
+
+No call here reaches a CUDA kernel (every argument set is invalid), so these
+run without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixed_precision_weight_row_b200 as mpw
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mpw.h")
+
+A16 = 0x10000          # fake, 16-byte aligned "device" addresses (never dereferenced)
+A16B = 0x20000
+ODD = 0x10001
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MPW_API\s+[\w\s\*]+?\b(mpw_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("mpw_quantize_pack", "mpw_unpack", "mpw_dequantize", "mpw_qlinear",
+                 "mpw_qlinear_path", "mpw_recipe_run", "mpw_packed_row_bytes",
+                 "mpw_status_str", "mpw_version", "mpw_device_error"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(mpw.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    for st in range(0, 7):
+        assert mpw.status_str(st) and mpw.status_str(st) != "unknown status"
+    assert mpw.status_str(99) == "unknown status"
+
+
+@pytest.mark.parametrize("bits", list(range(4, 16)))
+def test_packed_row_bytes_matches_oracle(bits):
+    for K in (1, 2, 31, 32, 33, 127, 128, 129, 4096, 5120, 17408, 100001):
+        assert mpw.packed_row_bytes(K, bits) == oracle.packed_row_bytes(K, bits)
+
+
+def test_packed_row_bytes_invalid():
+    assert mpw.packed_row_bytes(10, 3) == 0
+    assert mpw.packed_row_bytes(10, 16) == 0
+    assert mpw.packed_row_bytes(0, 8) == 0
+    assert mpw.packed_row_bytes(-5, 8) == 0
+
+
+def test_quantize_pack_validation():
+    L = mpw.lib
+    assert L.mpw_quantize_pack(A16, 4, 4, 3, A16B, A16, 0, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    assert L.mpw_quantize_pack(A16, 4, 4, 16, A16B, A16, 0, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    assert L.mpw_quantize_pack(0, 4, 4, 5, A16B, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_quantize_pack(A16, 4, 4, 5, 0, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_quantize_pack(A16, 4, 4, 5, A16B, 0, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_quantize_pack(A16, 0, 4, 5, A16B, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_quantize_pack(A16, 4, 0, 5, A16B, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_quantize_pack(A16, -1, 4, 5, A16B, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_quantize_pack(A16, 4, 4, 5, A16B + 8, A16, 0, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_quantize_pack(A16 + 2, 4, 4, 5, A16B, A16, 0, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_quantize_pack(A16, 4, 4, 5, A16B, A16, ODD, 0) == mpw.MPW_E_MISALIGNED
+
+
+def test_unpack_and_dequantize_validation():
+    L = mpw.lib
+    assert L.mpw_unpack(A16, 4, 4, 2, A16B, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    assert L.mpw_unpack(0, 4, 4, 5, A16B, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_unpack(A16, 4, 4, 5, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_unpack(A16 + 4, 4, 4, 5, A16B, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_unpack(A16, 4, 4, 5, ODD, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_dequantize(A16, A16B, 4, 4, 17, A16, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    assert L.mpw_dequantize(A16, 0, 4, 4, 5, A16, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_dequantize(A16, A16B, 4, 0, 5, A16, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_dequantize(A16, A16B + 1, 4, 4, 5, A16, 0) == mpw.MPW_E_MISALIGNED
+
+
+def test_qlinear_validation():
+    L = mpw.lib
+    assert L.mpw_qlinear(A16, A16B, A16, 3, 1, 4, 4, A16, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    assert L.mpw_qlinear(0, A16B, A16, 5, 1, 4, 4, A16, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear(A16, A16B, A16, 5, 0, 4, 4, A16, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear(A16, A16B, A16, 5, 1, 0, 4, A16, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear(A16, A16B, A16, 5, 1, 4, 0, A16, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear(A16, A16B, A16, 5, 1, 4, 4, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear(A16, A16B + 8, A16, 5, 1, 4, 4, A16, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_qlinear(ODD, A16B, A16, 5, 1, 4, 4, A16, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_qlinear_path(A16, A16B, A16, 5, 1, 4, 4, A16, 7, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_path(A16, A16B, A16, 5, 1, 4, 4, A16, -1, 0) == mpw.MPW_E_INVALID_ARG
+
+
+def _layers(*specs):
+    arr = (mpw._Linear * len(specs))()
+    for i, s in enumerate(specs):
+        arr[i] = mpw._Linear(*s)
+    return arr
+
+
+def test_recipe_run_validation():
+    L = mpw.lib
+    slots = (ctypes.c_void_p * 3)(A16, A16B, A16 + 0x100)
+    good = (A16, A16B, 8, 8, 6, 0, 1, 0)
+    assert L.mpw_recipe_run(_layers(good), 0, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_run(_layers(good), 1, slots, 3, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_run(_layers(good), 1, slots, 3, 33, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_run(_layers((A16, A16B, 8, 8, 3, 0, 1, 0)), 1, slots, 3, 1, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    assert L.mpw_recipe_run(_layers((A16, A16B, 8, 8, 6, 0, 0, 0)), 1, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_run(_layers((A16, A16B, 8, 8, 6, 0, 3, 0)), 1, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_run(_layers((A16, A16B, 8, 8, 6, -1, 1, 0)), 1, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_run(_layers((0, A16B, 8, 8, 6, 0, 1, 0)), 1, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_run(_layers((A16 + 4, A16B, 8, 8, 6, 0, 1, 0)), 1, slots, 3, 1, 0) == mpw.MPW_E_MISALIGNED
+    # an invalid entry anywhere in the list rejects the whole call before any launch
+    assert L.mpw_recipe_run(_layers(good, (A16, A16B, 8, 0, 6, 1, 2, 0)), 2, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    nulls = (ctypes.c_void_p * 3)(A16, 0, A16B)
+    assert L.mpw_recipe_run(_layers(good), 1, nulls, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+
+
+def test_device_error_rejects_null():
+    assert mpw.lib.mpw_device_error(None) == mpw.MPW_E_INVALID_ARG
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+
+    W = torch.zeros((4, 8), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        mpw.quantize_pack(W, 5)
+    with pytest.raises(TypeError):
+        mpw.quantize_pack(W.double(), 5)
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "mixed_precision_weight_row_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".h", ".cuh")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
