@@ -314,6 +314,74 @@ def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup
             "d2h_bytes_per_step": M * N * 2, "ms_per_step": ms / steps}
 
 
+def measure_prefill(mpw, pk, reps=10):
+    """Tensor-core prefill GEMM, x 2048x5120 bf16 against the two weight shapes."""
+    import torch
+
+    import workloads as wl
+
+    c = wl.PREFILL
+    x = wl.gen_x(c["M"], 5120, c["x_seed"]).cuda()
+    out = []
+    for name, N, K in c["shapes"]:
+        W = wl.gen_weight_torch(N, K, c["sigma"], 11 + N)
+        for b in c["bits"]:
+            packed, scales = mpw.quantize_pack(W, b)
+            y = torch.empty((c["M"], N), dtype=torch.bfloat16, device="cuda")
+            for _ in range(3):
+                mpw.qlinear(x, packed, scales, b, y=y)
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                mpw.qlinear(x, packed, scales, b, y=y)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / reps
+            flops = 2.0 * c["M"] * N * K
+            tf = flops / (us * 1e-6) / 1e12
+            executed = tf * (2 if b > 9 else 1)
+            out.append({"shape": f"{name} {N}x{K}", "b": b, "us": round(us, 2), "TFLOPs": round(tf, 1),
+                        "pct_bf16_peak": round(100 * tf / pk["bf16_tflops"], 2),
+                        "executed_mma_TFLOPs": round(executed, 1)})
+            del packed, scales, y
+        del W
+        torch.cuda.empty_cache()
+    assert mpw.device_error() == 0
+    return out
+
+
+def measure_recipe(mpw, pk, steps=10, warmup=3):
+    """448-matrix mixed-bit decode pass (M = 1) captured in one CUDA graph."""
+    import torch
+
+    import workloads as wl
+
+    shapes, bits, links = wl.recipe_shapes(), wl.recipe_bits(), wl.recipe_links()
+    layers = []
+    wbytes = 0
+    for i, ((layer, name, N, K), b, (si, so, nrm)) in enumerate(zip(shapes, bits, links)):
+        W = wl.gen_weight_torch(N, K, wl.RECIPE["sigma"], wl.recipe_weight_seed(i))
+        packed, scales = mpw.quantize_pack(W, b)
+        del W
+        layers.append(mpw.Linear(packed, scales, N, K, b, si, so, nrm))
+        wbytes += packed.numel() + scales.numel() * 4
+    slots = [torch.zeros((1, wl.SLOT_WIDTH[s]), dtype=torch.bfloat16, device="cuda") for s in range(8)]
+    slots[wl.SLOT_H].copy_(wl.gen_x(1, 5120, wl.RECIPE["x_seed"]).cuda())
+    g = graph_of(lambda: mpw.recipe_run(layers, slots, 1))
+    ms = time_graph(g, steps, warmup)
+    per = ms / steps
+    del g
+    res = {"matrices": len(layers), "weight_bytes": wbytes, "ms_per_token": round(per, 4),
+           "tokens_per_s": round(1e3 / per, 2), "weight_GBps": round(wbytes / (per * 1e-3) / 1e9, 1),
+           "pct_hbm": round(100 * wbytes / (per * 1e-3) / 1e9 / pk["hbm_gbs"], 2),
+           "launches_per_token": len(layers)}
+    del layers
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------------------
 # CPU baseline: the oracle, as it stands
 # ----------------------------------------------------------------------------
@@ -376,6 +444,46 @@ def run_reference(args, world, rank):
     return 0
 
 
+def run_case(args):
+    """A few launches of one kernel on one workload (for ncu captures)."""
+    import torch
+
+    import mixed_precision_weight_row_b200 as mpw
+    import workloads as wl
+
+    b, M = args.bits, args.M
+    if args.case in ("decode", "quantize"):
+        c = wl.DECODE
+        W = torch.from_numpy(wl.gen_weight(c["N"], c["K"], c["sigma"], c["w_seed"], c["outlier_frac"],
+                                           c["outlier_scale"])).cuda()
+    elif args.case in ("gate", "down"):
+        _, N, K = dict((n, (n, a, k)) for n, a, k in wl.MLP27B["shapes"])[args.case]
+        W = wl.gen_weight_torch(N, K, wl.MLP27B["sigma"], 17 + N)
+    elif args.case == "prefill":
+        _, N, K = wl.PREFILL["shapes"][0]
+        W = wl.gen_weight_torch(N, K, wl.PREFILL["sigma"], 11 + N)
+        M = wl.PREFILL["M"]
+    if args.case == "recipe":
+        shapes, bits, links = wl.recipe_shapes(1), wl.recipe_bits()[:7], wl.recipe_links(1)
+        layers = []
+        for i, ((_, _, N, K), bb, (si, so, nrm)) in enumerate(zip(shapes, bits, links)):
+            packed, scales = mpw.quantize_pack(wl.gen_weight_torch(N, K, 0.02, wl.recipe_weight_seed(i)), bb)
+            layers.append(mpw.Linear(packed, scales, N, K, bb, si, so, nrm))
+        slots = [torch.zeros((1, wl.SLOT_WIDTH[s]), dtype=torch.bfloat16, device="cuda") for s in range(8)]
+        for _ in range(args.launches):
+            mpw.recipe_run(layers, slots, 1)
+    elif args.case == "quantize":
+        for _ in range(args.launches):
+            mpw.quantize_pack(W, b)
+    else:
+        packed, scales = mpw.quantize_pack(W, b)
+        x = wl.gen_x(M, W.shape[1], 1).cuda()
+        for _ in range(args.launches):
+            mpw.qlinear(x, packed, scales, b)
+    torch.cuda.synchronize()
+    return 0
+
+
 def decode_config(args, pool):
     return {"workload": "decode GEMV sweep: W 4096x4096 ~N(0,0.02^2) + 0.1% outliers x20, "
                         f"b={HEADLINE_BITS}, x bf16 M=1",
@@ -393,6 +501,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--case", choices=["decode", "gate", "down", "prefill", "recipe", "quantize"],
+                    default=None, help="profiling target: run a few launches of one kernel, print nothing")
+    ap.add_argument("--bits", type=int, default=HEADLINE_BITS, help="bit width for --case")
+    ap.add_argument("--M", type=int, default=1, help="tokens for --case")
+    ap.add_argument("--launches", type=int, default=5, help="launches for --case")
     ap.add_argument("--quick", action="store_true",
                     help="headline and e2e only (no sweep, extras or CPU baseline)")
     args = ap.parse_args(argv)
@@ -400,6 +513,8 @@ def main(argv=None):
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.case is not None:
+        return run_case(args)
 
     import numpy as np
     import torch
@@ -477,6 +592,8 @@ def main(argv=None):
             del Wm
             torch.cuda.empty_cache()
         extras["mlp27b"] = mlp
+        extras["prefill"] = measure_prefill(mpw, pk)
+        extras["recipe"] = measure_recipe(mpw, pk)
 
     # ---- e2e: the public call with host buffers ----
     packed_h = pool.packed[0].cpu().pin_memory()

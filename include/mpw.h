@@ -142,9 +142,11 @@ MPW_API mpw_status mpw_qlinear_path(const uint16_t* x, const uint8_t* packed,
  *   packed, scales, N, K, bits  the quantized matrix (device pointers).
  *   in_slot   index of the slot holding x [M, K] (bf16).
  *   out_slot  index of the slot receiving y [M, N] (bf16).
- *   norm_input  if nonzero, the linear reads rms(x) instead of x, where
- *             rms(v) = bf16(v / sqrt(mean(v^2) + 1e-6)) per row, evaluated in
- *             fp32.  The normalised input is not written back.
+ *   norm_input  if nonzero, the linear reads the RMS-normalised input:
+ *             y[m, n] = bf16(s_n * r_m * sum_k x[m, k] q[n, k]) with
+ *             r_m = 1 / sqrt(mean_k x[m, k]^2 + 1e-6), evaluated in fp32 (the
+ *             normalisation is a per-token scale of the product; x itself is
+ *             not modified).
  */
 typedef struct mpw_linear {
   const uint8_t* packed;

@@ -68,6 +68,19 @@ cudaError_t ensure_smem_attr(const void* kernel, size_t bytes) {
   return cudaSuccess;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
 int32_t* device_error_word() {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;

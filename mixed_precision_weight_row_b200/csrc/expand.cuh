@@ -1,0 +1,184 @@
+// Code expansion for the tensor-core decode kernels: one 32-code group of a
+// packed row (B words) -> exact bf16 values in MMA fragment order.
+//
+// DynaQuant, "Custom kernel architecture": packed N-bit weights are expanded
+// in registers to a tensor-core format.  The schemes (all exact):
+//   * b = 4: the nibbles of codes k and k+4 sit 16 bits apart in a packed
+//     word, so one shift and one LOP3 give two bf16 values 128 + u'
+//     (u' = offset-binary code, OR-ed into the mantissa of 128.0);
+//   * b = 8: likewise for the low and the high nibbles of bytes k and k+2;
+//     q = 16*hi + lo, both parts fed to the same accumulator;
+//   * b = 5..7: codes k and k+1 are brought to bits 0 and 16 with one funnel
+//     shift, one shift and two LOP3s;
+//   * b >= 9: the offset-binary code is split into 7-bit fields (weights 1,
+//     128, 16384), each exact in bf16, one MMA per field.
+// A bf16x2 FMA on the FMA pipe removes the 128 offset and applies the field
+// weight, so every A operand is the exact code value.  The order of k inside
+// a 16-wide MMA step is free; x fragments are permuted to match.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace mpw {
+namespace dec {
+
+enum Scheme { kNib4, kNib8, kAdj1, kAdjSplit };
+
+template <int B>
+struct Exp {
+  static constexpr Scheme scheme = B == 4 ? kNib4 : (B == 8 ? kNib8 : (B <= 7 ? kAdj1 : kAdjSplit));
+  static constexpr int parts = B == 4 ? 1 : (B == 8 ? 2 : (B <= 7 ? 1 : (B <= 14 ? 2 : 3)));
+};
+
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t mul, uint32_t add) {
+  __nv_bfloat162 r = __hfma2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                             *reinterpret_cast<const __nv_bfloat162*>(&mul),
+                             *reinterpret_cast<const __nv_bfloat162*>(&add));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// bf16 bit patterns used below (exact values)
+constexpr uint32_t bf16_bits_of(int v) {
+  // v is an integer with at most 8 significant bits and |v| < 2^24 (exact in bf16)
+  if (v == 0) return 0u;
+  uint32_t s = v < 0 ? 0x8000u : 0u;
+  uint32_t a = static_cast<uint32_t>(v < 0 ? -v : v);
+  int e = 0;
+  while ((a >> e) > 1) ++e;                 // 2^e <= a < 2^(e+1)
+  uint32_t mant = e >= 7 ? (a >> (e - 7)) & 0x7Fu : (a << (7 - e)) & 0x7Fu;
+  return s | (static_cast<uint32_t>(127 + e) << 7) | mant;
+}
+constexpr uint32_t pair_of(int v) { return bf16_bits_of(v) | (bf16_bits_of(v) << 16); }
+
+// Pair of fields of codes c and c+1 (adjacent in the stream) starting at bit
+// offset f0 within each code, nb bits wide, as bf16 values 128 + field (with
+// the bits of `flip` XOR-ed into each field).  t holds code c at bit 0 and
+// code c+1 at bit B.
+// One LOP3: (a & b) ^ c.
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+// Low half from a, high half from b (one PRMT).
+__device__ __forceinline__ uint32_t merge_halves(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, 0x7610;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+template <int B, int F0, int NB, uint32_t FLIP>
+__device__ __forceinline__ uint32_t adj_pair(uint32_t t) {
+  const uint32_t a = F0 == 0 ? t : (t >> F0);
+  constexpr int sh = 16 - B - F0;  // where code c+1's field must move to reach bit 16
+  // a left shift is a multiply, which the FMA pipe can take off the ALU pipe
+  const uint32_t b = sh >= 0 ? (t * (1u << (sh >= 0 ? sh : 0))) : (t >> (sh < 0 ? -sh : 0));
+  constexpr uint32_t fm = ((1u << NB) - 1u) | (((1u << NB) - 1u) << 16);
+  constexpr uint32_t xm = 0x43004300u | FLIP | (FLIP << 16);
+  return and_xor(merge_halves(a, b), fm, xm);
+}
+
+// t = bits [o, o+32) of the group's words (code-aligned window)
+template <int B>
+__device__ __forceinline__ uint32_t window(const uint32_t (&w)[B + 1], int o) {
+  const int i = o >> 5, r = o & 31;
+  return r == 0 ? w[i] : __funnelshift_r(w[i], w[i + 1], r);
+}
+
+// Expands one 32-code group (B words) into parts x 16 bf16x2 registers; pair
+// p feeds MMA step p/2 (low / high k half).  All values are exact integers.
+template <int B>
+__device__ __forceinline__ void expand_group(const uint32_t (&w)[B + 1], uint32_t (&v)[Exp<B>::parts][16]) {
+  constexpr Scheme S = Exp<B>::scheme;
+  if constexpr (S == kNib4) {
+    // word i: codes 8i..8i+7; pair p = 4i+j = (code 8i+j, code 8i+j+4)
+    const uint32_t off = pair_of(-136);  // -(128 + 8)
+    const uint32_t one = pair_of(1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t r = ((w[i] >> (4 * j)) & 0x000F000Fu) ^ 0x43084308u;
+        v[0][4 * i + j] = bf2_fma(r, one, off);
+      }
+  } else if constexpr (S == kNib8) {
+    // word i: codes 4i..4i+3 (bytes); pair p = 2i+j = (code 4i+j, code 4i+j+2)
+    // q = 16*hi + lo with lo = low nibble (0..15), hi = high nibble (signed)
+    const uint32_t one = pair_of(1), m128 = pair_of(-128);
+    const uint32_t sixteen = pair_of(16), m2176 = pair_of(-2176);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t lo = ((w[i] >> (8 * j)) & 0x000F000Fu) | 0x43004300u;
+        const uint32_t hi = ((w[i] >> (8 * j + 4)) & 0x000F000Fu) ^ 0x43084308u;
+        v[0][2 * i + j] = bf2_fma(lo, one, m128);        // lo
+        v[1][2 * i + j] = bf2_fma(hi, sixteen, m2176);   // 16 * hi
+      }
+  } else if constexpr (S == kAdj1) {
+    constexpr int Q1 = 1 << (B - 1);
+    const uint32_t one = pair_of(1), off = pair_of(-(128 + Q1));
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      const uint32_t t = window<B>(w, 2 * p * B);
+      v[0][p] = bf2_fma(adj_pair<B, 0, B, (1u << (B - 1))>(t), one, off);
+    }
+  } else {
+    // offset-binary u' = u ^ 2^(B-1) split into 7-bit fields
+    const uint32_t one = pair_of(1), m128 = pair_of(-128);
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      const uint32_t t = window<B>(w, 2 * p * B);
+      v[0][p] = bf2_fma(adj_pair<B, 0, 7, 0u>(t), one, m128);  // lo7
+      if constexpr (B <= 14) {
+        // 128 * (mid - 2^(B-8)); the sign flip of u' lands in this field
+        constexpr int NB = B - 7;
+        v[1][p] = bf2_fma(adj_pair<B, 7, NB, (1u << (NB - 1))>(t), pair_of(128),
+                          pair_of(-128 * (128 + (1 << (B - 8)))));
+      } else {
+        v[1][p] = bf2_fma(adj_pair<B, 7, 7, 0u>(t), pair_of(128), pair_of(-128 * 128));
+        // top bit (with the flip): 16384 * (top - 1)
+        v[2][p] = bf2_fma(adj_pair<B, 14, 1, 1u>(t), pair_of(16384), pair_of(-16384 * 129));
+      }
+    }
+  }
+}
+
+// Permutes the raw x pairs (x[2m], x[2m+1]) of a group into the k order of
+// the expansion scheme.
+template <int B>
+__device__ __forceinline__ void permute_x(uint32_t (&xw)[16]) {
+  constexpr Scheme S = Exp<B>::scheme;
+  if constexpr (S == kNib4) {
+    uint32_t o[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        o[4 * i + j] = __byte_perm(xw[4 * i + (j >> 1)], xw[4 * i + 2 + (j >> 1)], (j & 1) ? 0x7632 : 0x5410);
+#pragma unroll
+    for (int p = 0; p < 16; ++p) xw[p] = o[p];
+  } else if constexpr (S == kNib8) {
+    uint32_t o[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) o[2 * i + j] = __byte_perm(xw[2 * i], xw[2 * i + 1], j ? 0x7632 : 0x5410);
+#pragma unroll
+    for (int p = 0; p < 16; ++p) xw[p] = o[p];
+  }
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+}  // namespace dec
+}  // namespace mpw

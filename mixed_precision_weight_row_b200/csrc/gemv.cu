@@ -5,23 +5,31 @@
 // saving in bytes is the speedup because the layer is bandwidth-bound
 // (quantization tutorial, closing note: decode is memory-bound).
 //
-// Work layout.  A warp owns R consecutive weight rows at a time.  Lane l walks
-// the row in groups of 32 codes (g = l, l+32, ...); one group of one row is
-// exactly B 32-bit words of the packed stream, so the warp reads 128*B
-// contiguous bytes per row per step.  Codes are expanded with one funnel
-// shift and one LOP3 each: the b-bit two's-complement field, with its sign
-// bit flipped, is OR-ed into the mantissa of 2^23, and one FADD removes the
-// 2^23 + 2^(b-1) offset, which gives the code as an exact fp32 integer.
-// x lives in shared memory as fp32, transposed so that lane l's eight float4
-// loads for its group are conflict-free and shared by the R rows.  Partial sums
-// use four accumulators per (row, token) and a final warp reduction; the row
-// scale is applied once, after the sum.
+// Code expansion (both kernels): one 32-code group of one row is exactly B
+// 32-bit words of the packed stream.  A code is isolated with one funnel
+// shift; its b-bit two's-complement field, sign bit flipped, is OR-ed into
+// the mantissa of 2^23 (one LOP3) and one FADD removes 2^23 + 2^(b-1), which
+// leaves the code as an exact fp32 integer.  Products accumulate in fp32 (four
+// partial sums per row and token); the row scale is applied once, after the
+// sum.
 //
-// CTAs are persistent (grid = min(tasks, resident CTAs)); x is staged once per
-// CTA when it fits in shared memory, else per K-chunk.
+// gemv_xreg_kernel (K <= 32768, the decode shapes): lane l of warp w owns the
+// group g = 32w + l of K for the whole kernel, so its 32 x values stay in
+// registers.  A CTA (ceil(K/32) lanes) walks a contiguous range of rows in
+// batches of 4, double-buffering the next batch's packed words in registers
+// (vector loads, streaming cache hint) while it computes the current one;
+// per-row partials are reduced with warp shuffles and one shared-memory pass.
+//
+// gemv_generic_kernel (any K): warps own rows, lanes walk the row; x is staged
+// in shared memory (per K-chunk when it does not fit).
+//
+// With norm_input the output is scaled by r_m = 1 / sqrt(mean_k x^2 + 1e-6)
+// (fp32, one fixed reduction order per kernel) after the dot product.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <cstdlib>
 
 #include "mpw_internal.h"
 
@@ -75,7 +83,6 @@ __device__ __forceinline__ void stage_x(float* xs, const uint16_t* __restrict__ 
       float v = 0.0f;
       if (t < mt && k < K) {
         v = bf16_bits_to_float(__ldg(src + k));
-        if (NORM) v = __bfloat162float(__float2bfloat16_rn(v * inv_rms[t]));
       }
       dst[xs_index(idx >> 5, idx & 31)] = v;
     }
@@ -109,7 +116,7 @@ __device__ void token_inv_rms(const uint16_t* __restrict__ x, int ldx, int mt, i
 
 template <int B, int R, int MT, bool NORM>
 __global__ void __launch_bounds__(kThreads)
-gemv_kernel(const uint16_t* __restrict__ x, int mt, const uint8_t* __restrict__ packed,
+gemv_generic_kernel(const uint16_t* __restrict__ x, int mt, const uint8_t* __restrict__ packed,
             const float* __restrict__ scales, int N, int K, int rw, uint16_t* __restrict__ y,
             int gc, int num_tasks) {
   extern __shared__ __align__(16) float xs[];
@@ -185,7 +192,7 @@ gemv_kernel(const uint16_t* __restrict__ x, int mt, const uint8_t* __restrict__ 
         float v = (acc[r][t][0] + acc[r][t][1]) + (acc[r][t][2] + acc[r][t][3]);
         v = warp_sum(v);
         if (lane == 0 && n < N && t < mt) {
-          const float outv = v * __ldg(scales + n);
+          const float outv = v * __ldg(scales + n) * (NORM ? inv_rms[t] : 1.0f);
           y[static_cast<size_t>(t) * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(outv));
         }
       }
@@ -194,7 +201,7 @@ gemv_kernel(const uint16_t* __restrict__ x, int mt, const uint8_t* __restrict__ 
 }
 
 template <int B, int R, int MT, bool NORM>
-cudaError_t run_gemv(const uint16_t* x, int mt, const uint8_t* packed, const float* scales, int N,
+cudaError_t run_gemv_generic(const uint16_t* x, int mt, const uint8_t* packed, const float* scales, int N,
                      int K, uint16_t* y, cudaStream_t stream) {
   const int rw = static_cast<int>(row_words(K, B));
   const int G = (K + 31) / 32;
@@ -202,7 +209,7 @@ cudaError_t run_gemv(const uint16_t* x, int mt, const uint8_t* packed, const flo
   int gc = static_cast<int>(kXSmemBudget / (static_cast<size_t>(MT) * 32 * 4)) / 32 * 32;
   if (gc > g_round) gc = g_round;
   const size_t smem = static_cast<size_t>(MT) * gc * 32 * 4;
-  auto kern = gemv_kernel<B, R, MT, NORM>;
+  auto kern = gemv_generic_kernel<B, R, MT, NORM>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kXSmemBudget);
   if (e != cudaSuccess) return e;
   const int rows_per_task = kWarps * R;
@@ -217,21 +224,214 @@ cudaError_t run_gemv(const uint16_t* x, int mt, const uint8_t* packed, const flo
   return cudaGetLastError();
 }
 
+
+// ---------------------------------------------------------------------------
+// x in registers, persistent row ranges
+// ---------------------------------------------------------------------------
+
+// Rows per batch: two batches of packed words plus the x slice must fit the
+// registers that __launch_bounds__ leaves (96 per thread when 17 warps share
+// the four SM sub-partitions); the thresholds keep every width spill-free.
+template <int B, int MT>
+constexpr int rows_per_batch() {
+  return (8 * (B + 1) + 32 * MT <= 88) ? 4 : ((4 * (B + 1) + 32 * MT <= 80) ? 2 : 1);
+}
+constexpr int kXregMaxThreads = 544;  // K <= 17408
+
+template <int B>
+__device__ __forceinline__ void load_words(const uint32_t* __restrict__ p, bool full, int avail,
+                                           uint32_t (&w)[B + 1]) {
+  if (full) {
+    if constexpr (B % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < B / 4; ++i) {
+        const uint4 v = __ldcs(reinterpret_cast<const uint4*>(p) + i);
+        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+      }
+    } else if constexpr (B % 2 == 0) {
+#pragma unroll
+      for (int i = 0; i < B / 2; ++i) {
+        const uint2 v = __ldcs(reinterpret_cast<const uint2*>(p) + i);
+        w[2 * i] = v.x; w[2 * i + 1] = v.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < B; ++i) w[i] = __ldcs(p + i);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < B; ++i) w[i] = i < avail ? __ldcs(p + i) : 0u;
+  }
+  w[B] = 0u;
+}
+
+template <int B, int MT, bool NORM>
+__global__ void __launch_bounds__(kXregMaxThreads, 1)
+gemv_xreg_kernel(const uint16_t* __restrict__ x, int mt, const uint8_t* __restrict__ packed,
+                 const float* __restrict__ scales, int N, int K, int rw, uint16_t* __restrict__ y) {
+  constexpr int kRB = rows_per_batch<B, MT>();
+  __shared__ float part[2][kRB][MT][32];
+  __shared__ float red[MT][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int G = (K + 31) >> 5;
+  const int g = warp * 32 + lane;
+  const bool gact = g < G;
+  const int avail = gact ? min(B, rw - g * B) : 0;   // words of this group inside the row
+  const bool full = avail == B;
+
+  const int r_begin = static_cast<int>((static_cast<int64_t>(N) * blockIdx.x) / gridDim.x);
+  const int r_end = static_cast<int>((static_cast<int64_t>(N) * (blockIdx.x + 1)) / gridDim.x);
+  const uint32_t* base = reinterpret_cast<const uint32_t*>(packed) + static_cast<size_t>(g) * B;
+
+  // first batch of packed words goes out before x is touched
+  uint32_t wa[kRB][B + 1], wb[kRB][B + 1];
+#pragma unroll
+  for (int i = 0; i < kRB; ++i) {
+    const int n = r_begin + i;
+    if (n < r_end && avail > 0) load_words<B>(base + static_cast<size_t>(n) * rw, full, avail, wa[i]);
+    else {
+#pragma unroll
+      for (int q = 0; q <= B; ++q) wa[i][q] = 0u;
+    }
+  }
+
+  // this lane's slice of x, as fp32
+  float xr[MT][32];
+#pragma unroll
+  for (int t = 0; t < MT; ++t) {
+    const uint16_t* xt = x + static_cast<size_t>(t) * K + static_cast<size_t>(g) * 32;
+    const bool vec = gact && t < mt && (g + 1) * 32 <= K && (reinterpret_cast<uintptr_t>(xt) & 15) == 0;
+    if (vec) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(xt) + i);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          xr[t][8 * i + 2 * c] = __uint_as_float(u[c] << 16);
+          xr[t][8 * i + 2 * c + 1] = __uint_as_float(u[c] & 0xffff0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int k = g * 32 + j;
+        xr[t][j] = (gact && t < mt && k < K) ? bf16_bits_to_float(__ldg(xt + j)) : 0.0f;
+      }
+    }
+  }
+  float inv[MT];
+#pragma unroll
+  for (int t = 0; t < MT; ++t) inv[t] = 1.0f;
+  if (NORM) {
+    // 1 / sqrt(mean(x^2) + 1e-6) per token, same reduction order in every CTA
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      float ss = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ss = fmaf(xr[t][j], xr[t][j], ss);
+      ss = warp_sum(ss);
+      if (lane == 0) red[t][warp] = ss;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      float tot = 0.0f;
+      for (int w = 0; w < nwarps; ++w) tot += red[t][w];
+      inv[t] = 1.0f / sqrtf(tot / static_cast<float>(K) + 1e-6f);
+    }
+  }
+
+  auto compute = [&](const uint32_t (&w)[kRB][B + 1], int r0, int par) {
+#pragma unroll
+    for (int i = 0; i < kRB; ++i) {
+      float acc[MT][4];
+#pragma unroll
+      for (int t = 0; t < MT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float q = code_f32<B>(w[i], j);
+#pragma unroll
+        for (int t = 0; t < MT; ++t) acc[t][j & 3] = fmaf(xr[t][j], q, acc[t][j & 3]);
+      }
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const float v = warp_sum((acc[t][0] + acc[t][1]) + (acc[t][2] + acc[t][3]));
+        if (lane == 0) part[par][i][t][warp] = v;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < kRB * MT) {
+      const int i = threadIdx.x / MT, t = threadIdx.x % MT;
+      const int n = r0 + i;
+      if (n < r_end && t < mt) {
+        float v = 0.0f;
+        for (int w = 0; w < nwarps; ++w) v += part[par][i][t][w];
+        const float sc = __ldg(scales + n) * (NORM ? inv[t] : 1.0f);
+        y[static_cast<size_t>(t) * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v * sc));
+      }
+    }
+  };
+  auto load_batch = [&](uint32_t (&w)[kRB][B + 1], int r0) {
+#pragma unroll
+    for (int i = 0; i < kRB; ++i) {
+      const int n = r0 + i;
+      if (n < r_end && avail > 0) load_words<B>(base + static_cast<size_t>(n) * rw, full, avail, w[i]);
+    }
+  };
+
+  for (int r = r_begin; r < r_end; r += 2 * kRB) {
+    load_batch(wb, r + kRB);
+    compute(wa, r, 0);
+    load_batch(wa, r + 2 * kRB);
+    if (r + kRB < r_end) compute(wb, r + kRB, 1);
+  }
+}
+
+template <int B, int MT, bool NORM>
+cudaError_t run_gemv_xreg(const uint16_t* x, int mt, const uint8_t* packed, const float* scales, int N,
+                          int K, uint16_t* y, cudaStream_t stream) {
+  const int rw = static_cast<int>(row_words(K, B));
+  const int G = (K + 31) / 32;
+  const int threads = (G + 31) / 32 * 32;
+  auto kern = gemv_xreg_kernel<B, MT, NORM>;
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  int grid = per_sm * device_info().num_sms;
+  if (grid > N) grid = N;
+  kern<<<grid, threads, 0, stream>>>(x, mt, packed, scales, N, K, rw, y);
+  return cudaGetLastError();
+}
+
 template <int B>
 cudaError_t gemv_bits(const uint16_t* x, int64_t M, const uint8_t* packed, const float* scales,
                       int64_t N, int64_t K, uint16_t* y, bool norm, cudaStream_t stream) {
+  const bool xreg = K <= kXregMaxThreads * 32;  // one group per lane
   // passes over the tokens: 2 at a time, a last single one if M is odd
   for (int64_t m0 = 0; m0 < M; m0 += 2) {
     const int mt = static_cast<int>(M - m0 >= 2 ? 2 : 1);
     const uint16_t* xp = x + m0 * K;
     uint16_t* yp = y + m0 * N;
+    const int n = static_cast<int>(N), k = static_cast<int>(K);
     cudaError_t e;
-    if (mt == 2)
-      e = norm ? run_gemv<B, 2, 2, true>(xp, mt, packed, scales, static_cast<int>(N), static_cast<int>(K), yp, stream)
-               : run_gemv<B, 2, 2, false>(xp, mt, packed, scales, static_cast<int>(N), static_cast<int>(K), yp, stream);
-    else
-      e = norm ? run_gemv<B, 4, 1, true>(xp, mt, packed, scales, static_cast<int>(N), static_cast<int>(K), yp, stream)
-               : run_gemv<B, 4, 1, false>(xp, mt, packed, scales, static_cast<int>(N), static_cast<int>(K), yp, stream);
+    if (xreg) {
+      if (mt == 2)
+        e = norm ? run_gemv_xreg<B, 2, true>(xp, mt, packed, scales, n, k, yp, stream)
+                 : run_gemv_xreg<B, 2, false>(xp, mt, packed, scales, n, k, yp, stream);
+      else
+        e = norm ? run_gemv_xreg<B, 1, true>(xp, mt, packed, scales, n, k, yp, stream)
+                 : run_gemv_xreg<B, 1, false>(xp, mt, packed, scales, n, k, yp, stream);
+    } else {
+      if (mt == 2)
+        e = norm ? run_gemv_generic<B, 2, 2, true>(xp, mt, packed, scales, n, k, yp, stream)
+                 : run_gemv_generic<B, 2, 2, false>(xp, mt, packed, scales, n, k, yp, stream);
+      else
+        e = norm ? run_gemv_generic<B, 4, 1, true>(xp, mt, packed, scales, n, k, yp, stream)
+                 : run_gemv_generic<B, 4, 1, false>(xp, mt, packed, scales, n, k, yp, stream);
+    }
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -242,6 +442,32 @@ cudaError_t gemv_bits(const uint16_t* x, int64_t M, const uint8_t* packed, const
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm_input,
                         cudaStream_t stream) {
+  // Tensor-core decode kernel in passes of up to 32 tokens (8 with norm_input).
+  // MPW_GEMV_KERNEL=mma selects the register-streaming variant (tuning aid).
+  static const bool use_mma = [] {
+    const char* e = getenv("MPW_GEMV_KERNEL");
+    return e != nullptr && e[0] == 'm';
+  }();
+  const int64_t pass = norm_input ? 8 : 32;
+  const int64_t m1 = M < pass ? M : pass;
+  const bool tma = !use_mma && gemv_tma_supported(m1, N, K, norm_input);
+  if (tma || gemv_mma_supported(m1, N, K, norm_input)) {
+    for (int64_t m0 = 0; m0 < M; m0 += pass) {
+      const int64_t mt = M - m0 < pass ? M - m0 : pass;
+      cudaError_t e = tma ? launch_gemv_tma(x + m0 * K, packed, scales, bits, mt, N, K, y + m0 * N, norm_input,
+                                            /*pdl=*/true, stream)
+                          : launch_gemv_mma(x + m0 * K, packed, scales, bits, mt, N, K, y + m0 * N, norm_input,
+                                            /*pdl=*/true, stream);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaGetLastError();
+  }
+  return launch_gemv_cuda_core(x, packed, scales, bits, M, N, K, y, norm_input, stream);
+}
+
+cudaError_t launch_gemv_cuda_core(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                                  int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm_input,
+                                  cudaStream_t stream) {
   switch (bits) {
     case 4: return gemv_bits<4>(x, M, packed, scales, N, K, y, norm_input, stream);
     case 5: return gemv_bits<5>(x, M, packed, scales, N, K, y, norm_input, stream);

@@ -3,6 +3,8 @@
 // argument before it calls them.  Each returns the cudaError_t of its launch.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -22,6 +24,12 @@ struct DeviceInfo {
 };
 const DeviceInfo& device_info();
 
+// cuTensorMapEncodeTiled from the driver (nullptr if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Device address of the library's device-side error word.
+int32_t* device_error_word();
+
 // Raises a kernel's dynamic shared-memory limit to `bytes` on the current
 // device (once per kernel and device).
 cudaError_t ensure_smem_attr(const void* kernel, size_t bytes);
@@ -35,10 +43,30 @@ cudaError_t launch_unpack(const uint8_t* packed, int64_t N, int64_t K, int bits,
 cudaError_t launch_dequantize(const uint8_t* packed, const float* scales, int64_t N,
                               int64_t K, int bits, float* W_hat, cudaStream_t stream);
 
-// gemv.cu: y[M, N] for any M, in passes of at most kGemvMaxTokens rows of x.
+// gemv.cu: decode linear y[M, N] for any M (tensor-core kernel in passes of
+// 32 tokens; CUDA-core kernels for shapes it does not take).
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* scales,
                         int bits, int64_t M, int64_t N, int64_t K, uint16_t* y,
                         bool norm_input, cudaStream_t stream);
+// The CUDA-core decode kernels alone (x in registers for K <= 17408, else x
+// staged in shared memory), in passes of two tokens.
+cudaError_t launch_gemv_cuda_core(const uint16_t* x, const uint8_t* packed, const float* scales,
+                                  int bits, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                  bool norm_input, cudaStream_t stream);
+
+// gemv_mma.cu: decode linear on register-fed tensor cores for M <= 32
+// (M <= 8 with norm_input); pdl = launch with programmatic dependent launch.
+bool gemv_mma_supported(int64_t M, int64_t N, int64_t K, bool norm);
+cudaError_t launch_gemv_mma(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                            int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, bool pdl,
+                            cudaStream_t stream);
+
+// gemv_tma.cu: decode linear with the packed stream staged by TMA in a
+// shared-memory ring (the default decode kernel for M <= 32).
+bool gemv_tma_supported(int64_t M, int64_t N, int64_t K, bool norm);
+cudaError_t launch_gemv_tma(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                            int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, bool pdl,
+                            cudaStream_t stream);
 
 // gemm.cu: tcgen05 prefill GEMM; returns cudaErrorNotSupported for shapes it
 // does not take (the caller then uses the GEMV path).

@@ -18,7 +18,8 @@ from .quant import (  # noqa: F401
     quality,
     quantize,
     quantize_pack,
-    rms_normalize_bf16,
+    qlinear_rms_ref,
+    rms_scale,
     row_scales,
     unpack,
     unpadded_row_bytes,

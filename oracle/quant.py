@@ -35,6 +35,9 @@ notes):
   computed in fp64 from the exact w_hat = q * s, and an output is accepted when
   |y - y_ref| <= 8e-3 * sum_k |x[m, k] * w_hat[n, k]| + 1e-6.
 * Non-finite weights are outside the method's domain: the oracle raises.
+* Recipe data flow (no page gives one): a linear flagged to read the
+  normalised input computes y = s_n * r_m * sum_k x[m, k] q[n, k] with
+  r_m = 1 / sqrt(mean_k x[m, k]^2 + 1e-6).
 """
 from __future__ import annotations
 
@@ -204,19 +207,22 @@ def check_qlinear(y_gpu, y_ref, bound):
 RMS_EPS = 1e-6
 
 
-def rms_normalize_bf16(v) -> np.ndarray:
-    """bf16(v / sqrt(mean(v^2) + 1e-6)) per row, evaluated in fp64.
+def rms_scale(v) -> np.ndarray:
+    """r_m = 1 / sqrt(mean_k(v[m, k]^2) + 1e-6) per row of v, in fp64.
 
-    The pages give no data flow between the linears of the recipe stack; this
-    normalisation keeps the chained pass in range (see the design notes).
-    Returned as float32 values that are exactly bf16 (round to nearest even).
+    The pages give no data flow between the linears of the recipe stack; a
+    linear that "reads rms(x)" computes y = s_n * r_m * sum_k x[m, k] q[n, k],
+    i.e. the normalisation is a per-token scale applied to the product (see
+    the design notes).  Returns shape [M, 1].
     """
-    import torch
-
     v = np.asarray(v, dtype=np.float64)
-    ms = np.mean(v ** 2, axis=-1, keepdims=True)
-    out = v / np.sqrt(ms + RMS_EPS)
-    return torch.from_numpy(out).to(torch.bfloat16).float().numpy()
+    return 1.0 / np.sqrt(np.mean(v ** 2, axis=-1, keepdims=True) + RMS_EPS)
+
+
+def qlinear_rms_ref(x, q: np.ndarray, s: np.ndarray):
+    """(y_ref, bound) for the linear of the rms-scaled input r_m * x[m, :]."""
+    x64 = np.asarray(x, dtype=np.float64) * rms_scale(x)
+    return qlinear_ref(x64, q, s)
 
 
 # ----------------------------------------------------------------------------

@@ -211,3 +211,57 @@ def test_quantize_then_qlinear_roundtrip(mpw):
         q, s = oracle.quantize(W, b)
         y_ref, bound = oracle.qlinear_ref(x.float().numpy(), q, s)
         assert oracle.check_qlinear(y.float().cpu().numpy(), y_ref, bound).all()
+
+
+# ----------------------------------------------------------------------------
+# tensor-core prefill GEMM
+# ----------------------------------------------------------------------------
+
+GEMM_SHAPES = [(33, 1, 8), (64, 40, 64), (256, 128, 128), (300, 200, 520), (513, 129, 1000), (40, 260, 4104)]
+
+
+@pytest.mark.parametrize("b", BITS)
+def test_qlinear_gemm_small(mpw, b):
+    rng = np.random.default_rng(3000 + b)
+    for M, N, K in GEMM_SHAPES:
+        W = rng.standard_normal((N, K)).astype(np.float32) * np.float32(0.02)
+        if N > 3:
+            W[2] = 0
+        x = workloads.gen_x(M, K, seed=M + K + b)
+        _check_qlinear(mpw, W, x, b, path="gemm")
+
+
+@pytest.mark.parametrize("b", [4, 8, 9, 10, 15])
+@pytest.mark.parametrize("M", [1, 16, 32])
+def test_qlinear_gemm_path_small_m(mpw, b, M):
+    rng = np.random.default_rng(4000 + b + M)
+    W = rng.standard_normal((150, 256)).astype(np.float32)
+    x = workloads.gen_x(M, 256, seed=M)
+    _check_qlinear(mpw, W, x, b, path="gemm")
+
+
+def test_qlinear_auto_routes_odd_k_to_gemv(mpw):
+    # K % 8 != 0 cannot be a TMA operand: auto falls back to the decode kernel
+    rng = np.random.default_rng(6)
+    W = rng.standard_normal((64, 301)).astype(np.float32)
+    x = workloads.gen_x(70, 301, seed=6)
+    _check_qlinear(mpw, W, x, 7)
+    with pytest.raises(mpw.MPWError):
+        _check_qlinear(mpw, W, x, 7, path="gemm")
+
+
+def test_gemm_extreme_codes(mpw):
+    # rows that hit +-Q everywhere and x of both signs: exercises the hi/lo split
+    rng = np.random.default_rng(8)
+    for b in (9, 10, 12, 15):
+        W = np.where(rng.random((128, 512)) < 0.5, -1.0, 1.0).astype(np.float32)
+        x = workloads.gen_x(256, 512, seed=b)
+        _check_qlinear(mpw, W, x, b, path="gemm")
+
+
+def test_gemm_device_error_word_clear(mpw):
+    rng = np.random.default_rng(10)
+    W = rng.standard_normal((128, 256)).astype(np.float32)
+    x = workloads.gen_x(64, 256, seed=1)
+    _check_qlinear(mpw, W, x, 6, path="gemm")
+    assert mpw.device_error() == 0

@@ -89,3 +89,22 @@ def test_mlp27b_workload_sampled(mpw, name, N, K, b):
         y_ref, bound = oracle.qlinear_ref(x.float().numpy(), q, s)
         ok = oracle.check_qlinear(y, y_ref, bound)
         assert ok.all(), f"M={M}: {(~ok).sum()} sampled outputs out of bound"
+
+
+@pytest.mark.parametrize("name,N,K", wl.PREFILL["shapes"], ids=["up", "o"])
+@pytest.mark.parametrize("b", wl.PREFILL["bits"])
+def test_prefill_workload_sampled(mpw, name, N, K, b):
+    torch = _t()
+    c = wl.PREFILL
+    W = wl.gen_weight(N, K, c["sigma"], c["w_seed"])
+    x = wl.gen_x(c["M"], K, c["x_seed"])
+    packed, scales = mpw.quantize_pack(torch.from_numpy(W).cuda(), b)
+    y = mpw.qlinear(x.cuda(), packed, scales, b)          # M = 2048 -> tensor-core GEMM
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(321)
+    rows = np.unique(np.concatenate([[0, 127, 128, N - 1], rng.choice(N, 124, replace=False)]))
+    q, s = oracle.quantize(W[rows], b)
+    y_ref, bound = oracle.qlinear_ref(x.float().numpy(), q, s)
+    ok = oracle.check_qlinear(y.float().cpu().numpy()[:, rows], y_ref, bound)
+    assert ok.all(), f"{(~ok).sum()} sampled outputs out of bound"
+    assert mpw.device_error() == 0

@@ -352,3 +352,25 @@ def test_bits_out_of_range_are_rejected():
         oracle.qmax(3)
     with pytest.raises(ValueError):
         oracle.qmax(16)
+
+
+def test_rms_scale_closed_forms():
+    # constant rows: mean(v^2) = c^2, so r = 1 / sqrt(c^2 + 1e-6)
+    v = np.array([[2.0] * 10, [-0.5] * 4 + [0.5] * 4, [0.0] * 3], dtype=object)
+    r0 = oracle.rms_scale(np.full((1, 10), 2.0))[0, 0]
+    assert abs(r0 - 1.0 / np.sqrt(4.0 + 1e-6)) < 1e-15
+    r1 = oracle.rms_scale(np.array([[-0.5, 0.5, -0.5, 0.5]]))[0, 0]
+    assert abs(r1 - 1.0 / np.sqrt(0.25 + 1e-6)) < 1e-15
+    r2 = oracle.rms_scale(np.zeros((1, 3)))[0, 0]
+    assert abs(r2 - 1000.0) < 1e-9
+    # the scaled row has mean square 1 up to the epsilon
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((3, 500)) * 7.0
+    xs = x * oracle.rms_scale(x)
+    assert np.allclose(np.mean(xs ** 2, axis=1), 1.0, atol=1e-6)
+    # the rms-scaled linear is the plain linear scaled per token
+    W = rng.standard_normal((6, 500)).astype(np.float32)
+    q, s = oracle.quantize(W, 7)
+    y1, _ = oracle.qlinear_rms_ref(x, q, s)
+    y0, _ = oracle.qlinear_ref(x, q, s)
+    assert np.allclose(y1, y0 * oracle.rms_scale(x), rtol=1e-12)

@@ -151,3 +151,38 @@ def special_rows(K: int, seed: int = 7) -> np.ndarray:
                rng.choice([-1.0, 1.0], size=K)).astype(np.float32)
     W[7, :] = rng.standard_normal(K).astype(np.float32)
     return W
+
+
+# ----------------------------------------------------------------------------
+# recipe stack data flow
+# ----------------------------------------------------------------------------
+
+# Activation slots of the chained decode pass.  The pages give no data flow
+# between the linears of a layer; this one follows a decoder layer's shape
+# (q/k/v read the hidden state, o reads the attention-side output, gate/up
+# read o's output, down reads up's output) with an RMS normalisation on every
+# linear's input after the first, which keeps 64 chained layers in range.
+SLOT_H, SLOT_Q, SLOT_K, SLOT_V, SLOT_O, SLOT_G, SLOT_U, SLOT_D = range(8)
+SLOT_WIDTH = {SLOT_H: 5120, SLOT_Q: 6144, SLOT_K: 1024, SLOT_V: 1024, SLOT_O: 5120,
+              SLOT_G: 17408, SLOT_U: 17408, SLOT_D: 5120}
+
+
+def recipe_links(layers: int = RECIPE_LAYERS):
+    """(in_slot, out_slot, norm_input) for every linear, in recipe order.
+
+    Layer 0's q/k/v read x0 (slot H) as is; later layers read the previous
+    layer's down output (slot D) normalised.
+    """
+    out = []
+    for layer in range(layers):
+        h = SLOT_H if layer == 0 else SLOT_D
+        hn = layer > 0
+        out += [(h, SLOT_Q, hn), (h, SLOT_K, hn), (h, SLOT_V, hn),
+                (SLOT_Q, SLOT_O, True), (SLOT_O, SLOT_G, True), (SLOT_O, SLOT_U, True),
+                (SLOT_U, SLOT_D, True)]
+    return out
+
+
+def recipe_weight_seed(index: int) -> int:
+    """Seed of the index-th matrix of the recipe stack."""
+    return 1000 * RECIPE["w_seed"] + 17 + index
