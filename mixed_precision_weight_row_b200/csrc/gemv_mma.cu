@@ -37,9 +37,10 @@
 // distributed shared memory into the cluster's first CTA, which applies the
 // row scale and writes bf16.  The packed words of the next two chunks of a
 // warp's slice and the next chunk's x fragments are in flight while the
-// current chunk is expanded.  Launches use programmatic dependent launch: the first chunk of
-// packed weights is requested before griddepcontrol.wait, so a chain of
-// linears streams weights while the previous kernel drains.
+// current chunk is expanded.  Launches use programmatic dependent launch:
+// each CTA allows its dependent launch as soon as it starts and waits for its
+// predecessor only before the first read of x, so in a chain of linears the
+// next kernel's CTAs are resident while this one drains.
 #include <cooperative_groups.h>
 #include <math.h>
 #include <cuda_bf16.h>
@@ -119,6 +120,9 @@ gemv_mma_kernel(const uint16_t* __restrict__ x, int M, const uint8_t* __restrict
   __shared__ float ss_red[kWarps][NS];
   __shared__ float cl_ss[8][NS];
 
+  // The next kernel in the stream may launch right away: it only reads its
+  // own weights until it passes griddepcontrol.wait.
+  asm volatile("griddepcontrol.launch_dependents;");
   cg::cluster_group cluster = cg::this_cluster();
   const int KC = static_cast<int>(cluster.num_blocks());
   const int cr = static_cast<int>(cluster.block_rank());
@@ -230,7 +234,6 @@ gemv_mma_kernel(const uint16_t* __restrict__ x, int M, const uint8_t* __restrict
   // everything above reads only the weights; x may still be being written by
   // the previous kernel in the stream
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;");
   if (n_main > 0) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) load_x_vec(px[nt], x0[nt]);

@@ -22,10 +22,10 @@
 // memory and distributed shared memory into the cluster's first CTA, which
 // applies the row scale (and the rms scale with norm_input) and writes bf16.
 //
-// Programmatic dependent launch: the producer's TMA loads read only W and are
-// issued before griddepcontrol.wait; the consumers wait before touching x or
-// y.  In a chain of linears the next layer's weights stream in while the
-// previous kernel drains.  Every mbarrier wait is bounded (2 s), after which
+// Programmatic dependent launch: every thread lets the next kernel launch at
+// once; the producer's TMA loads read only W and never wait, the consumers
+// wait (griddepcontrol.wait) before touching x or y.  In a chain of linears
+// the next layer's weights stream in while the previous kernel drains.  Every mbarrier wait is bounded (2 s), after which
 // the kernel records an error in the device error word and winds down.
 #include <cooperative_groups.h>
 #include <cuda.h>
@@ -98,6 +98,9 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t* __re
   __shared__ float ss_red[kCW][NS];
   __shared__ float cl_ss[8][NS];
 
+  // The next kernel in the stream may launch right away: it only streams its
+  // own weights until its consumers pass griddepcontrol.wait.
+  asm volatile("griddepcontrol.launch_dependents;");
   cg::cluster_group cluster = cg::this_cluster();
   const int KC = static_cast<int>(cluster.num_blocks());
   const int cr = static_cast<int>(cluster.block_rank());
@@ -143,11 +146,10 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t* __re
       // nothing may still be landing in shared memory when the CTA exits
       for (int s = max(0, issued - S); s < issued; ++s) ptx::mbar_wait(full(s % S), (s / S) & 1, err);
     }
-    asm volatile("griddepcontrol.launch_dependents;");
   } else {
     // ---------------- consumers ----------------
+    // x (and y) may belong to the previous kernel in the stream
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;");
     float acc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
