@@ -6,11 +6,14 @@ and the CPU-baseline leg of ``bench.py``; never by the library.
 from .quant import (  # noqa: F401
     MAX_BITS,
     MIN_BITS,
+    PAIR_GROUP,
     QLINEAR_ABS_TOL,
     QLINEAR_REL_TOL,
     check_qlinear,
     dequantize,
     pack,
+    pack_paired,
+    pair_halves,
     packed_row_bytes,
     qlinear_ref,
     qlinear_rows_ref,
@@ -22,5 +25,6 @@ from .quant import (  # noqa: F401
     rms_scale,
     row_scales,
     unpack,
+    unpack_paired,
     unpadded_row_bytes,
 )

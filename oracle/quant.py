@@ -155,6 +155,72 @@ def unpack(packed: np.ndarray, K: int, b: int) -> np.ndarray:
     return q.astype(np.int32)
 
 
+# ----------------------------------------------------------------------------
+# Paired-halves layout: a kernel-private re-ordering of the same bits.  No page
+# defines it; the decode kernels read it because a 32-bit word then holds two
+# codes 16 bits apart, the form in which they become one bf16x2 operand.
+# ----------------------------------------------------------------------------
+
+PAIR_GROUP = 32  # codes per group; K must be a multiple
+
+
+def _paired_check(K: int, b: int) -> None:
+    _check_bits(b)
+    if K < 1 or K % PAIR_GROUP != 0:
+        raise ValueError("the paired layout needs K to be a positive multiple of 32")
+
+
+def pack_paired(q: np.ndarray, b: int) -> np.ndarray:
+    """uint8[N, packed_row_bytes(K, b)] in the paired-halves layout.
+
+    Row n is cut into groups of 32 codes.  In group g the even codes
+    q[32g + 2i] (i = 0..15) form the stream E and the odd codes q[32g + 2i + 1]
+    the stream O; in each stream code i occupies bits [i*b, i*b + b), LSB
+    first, as b-bit two's complement, so each stream is b half-words of 16
+    bits.  Little-endian 32-bit word g*b + h of the row holds half-word h of E
+    in its low 16 bits and half-word h of O in its high 16 bits.  The bytes
+    after the last group are zero.  The row stride is the canonical one, and
+    the layout holds exactly the canonical bits, re-ordered.
+    """
+    q = np.asarray(q)
+    N, K = q.shape
+    _paired_check(K, b)
+    if np.any(np.abs(q) > qmax(b)):
+        raise ValueError("code outside +-Q")
+    G = K // PAIR_GROUP
+    u = (q.astype(np.int64) & ((1 << b) - 1)).astype(np.uint32).reshape(N, G, 16, 2)
+    # bits[n, g, stream, i*b + t] = bit t of code i of the stream
+    bits = ((u[..., None] >> np.arange(b, dtype=np.uint32)) & 1).astype(np.uint8)  # [N,G,16,2,b]
+    streams = bits.transpose(0, 1, 3, 2, 4).reshape(N, G, 2, b, 16)  # [N,G,stream,half-word,bit]
+    words = np.concatenate([streams[:, :, 0], streams[:, :, 1]], axis=3)  # [N,G,b,32]: E low, O high
+    out = np.zeros((N, packed_row_bytes(K, b) * 8), dtype=np.uint8)
+    out[:, : G * b * 32] = words.reshape(N, G * b * 32)
+    return np.packbits(out, axis=1, bitorder="little")
+
+
+def unpack_paired(packed: np.ndarray, K: int, b: int) -> np.ndarray:
+    """int32[N, K]: the codes held by a paired-halves row (inverse of
+    :func:`pack_paired`), sign-extended."""
+    packed = np.asarray(packed, dtype=np.uint8)
+    _paired_check(K, b)
+    N = packed.shape[0]
+    if packed.shape[1] != packed_row_bytes(K, b):
+        raise ValueError("row stride does not match K and b")
+    G = K // PAIR_GROUP
+    bits = np.unpackbits(packed, axis=1, bitorder="little")[:, : G * b * 32]
+    words = bits.reshape(N, G, b, 32)
+    streams = np.stack([words[..., :16], words[..., 16:]], axis=2)  # [N,G,stream,b,16]
+    codes_bits = streams.reshape(N, G, 2, 16, b).astype(np.int64)  # [N,G,stream,i,t]
+    u = (codes_bits << np.arange(b, dtype=np.int64)).sum(axis=4)  # [N,G,stream,i]
+    q = np.where(u >= (1 << (b - 1)), u - (1 << b), u)
+    return q.transpose(0, 1, 3, 2).reshape(N, K).astype(np.int32)
+
+
+def pair_halves(packed: np.ndarray, K: int, b: int) -> np.ndarray:
+    """Canonical packed rows re-ordered into the paired-halves layout."""
+    return pack_paired(unpack(packed, K, b), b)
+
+
 def quantize_pack(W: np.ndarray, b: int):
     """(packed uint8[N, rb], s float32[N]) -- the whole quantizer."""
     q, s = quantize(W, b)

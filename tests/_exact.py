@@ -103,3 +103,23 @@ def unpack_row_int(data: bytes, b: int, K: int):
         u = (acc >> (k * b)) & ((1 << b) - 1)
         out.append(u - (1 << b) if u >= (1 << (b - 1)) else u)
     return out
+
+
+def pack_paired_row_int(codes, b: int) -> bytes:
+    """Paired-halves row written with Python integers: per 32-code group, the
+    even codes form one integer stream and the odd codes another; each 32-bit
+    word takes 16 bits of each, low half from the even stream."""
+    assert len(codes) % 32 == 0
+    mask = (1 << b) - 1
+    words = []
+    for g0 in range(0, len(codes), 32):
+        even = 0
+        odd = 0
+        for i in range(16):
+            even += (codes[g0 + 2 * i] & mask) * 2 ** (i * b)
+            odd += (codes[g0 + 2 * i + 1] & mask) * 2 ** (i * b)
+        for h in range(b):
+            lo = (even // 2 ** (16 * h)) % 2 ** 16
+            hi = (odd // 2 ** (16 * h)) % 2 ** 16
+            words.append(lo + hi * 2 ** 16)
+    return b"".join(w.to_bytes(4, "little") for w in words)

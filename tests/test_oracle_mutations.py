@@ -25,6 +25,9 @@ def _run_pins():
     checks += [lambda b=b: pins.test_qlinear_against_fraction_triple_loop(b) for b in (5, 12)]
     checks += [lambda b=b: pins.test_packed_sizes(b) for b in (5, 7)]
     checks += [lambda b=b: pins.test_rounding_error_bound(b) for b in (4, 9)]
+    checks += [lambda b=b: pins.test_paired_matches_big_integer_packer(b) for b in (5, 8)]
+    checks += [lambda: pins.test_paired_b8_bytes_are_2x2_transposes(), lambda: pins.test_paired_b4_nibble_order()]
+    checks += [lambda b=b: pins.test_unpack_paired_inverts_pack_paired(b) for b in (7,)]
     for c in checks:
         try:
             c()
@@ -74,6 +77,10 @@ MUTANTS = {
     "unpack_without_sign_extension": lambda mp: _patch(mp, "unpack", lambda p, K, b: np.where(
         ORIG_UNPACK(p, K, b) < 0, ORIG_UNPACK(p, K, b) + (1 << b), ORIG_UNPACK(p, K, b)).astype(np.int32)),
     "qlinear_drops_scale": lambda mp: _patch(mp, "qlinear_ref", lambda x, q, s: ORIG_QLINEAR(x, q, np.ones_like(s))),
+    "paired_streams_swapped": lambda mp: _patch(mp, "pack_paired", lambda q, b: ORIG_PACK_PAIRED(
+        np.ascontiguousarray(q.reshape(q.shape[0], -1, 2)[:, :, ::-1].reshape(q.shape)), b)),
+    "paired_codes_adjacent_not_even_odd": lambda mp: _patch(mp, "pack_paired", lambda q, b: ORIG_PACK_PAIRED(
+        np.ascontiguousarray(q.reshape(q.shape[0], -1, 2, 16).transpose(0, 1, 3, 2).reshape(q.shape)), b)),
     "qlinear_transposed_codes": lambda mp: _patch(mp, "qlinear_ref", lambda x, q, s: ORIG_QLINEAR(
         x, np.ascontiguousarray(q[::-1]), s[::-1])),
 }
@@ -81,6 +88,7 @@ MUTANTS = {
 ORIG_PACK = oq.pack
 ORIG_UNPACK = oq.unpack
 ORIG_QLINEAR = oq.qlinear_ref
+ORIG_PACK_PAIRED = oq.pack_paired
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

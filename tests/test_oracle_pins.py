@@ -374,3 +374,79 @@ def test_rms_scale_closed_forms():
     y1, _ = oracle.qlinear_rms_ref(x, q, s)
     y0, _ = oracle.qlinear_ref(x, q, s)
     assert np.allclose(y1, y0 * oracle.rms_scale(x), rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# Paired-halves layout (kernel-private ordering of the packed bits)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("b", list(range(4, 16)))
+def test_paired_matches_big_integer_packer(b):
+    rng = np.random.default_rng(700 + b)
+    Q = oracle.qmax(b)
+    K = 96
+    q = rng.integers(-Q, Q + 1, size=(3, K)).astype(np.int32)
+    q[0, :32] = Q
+    q[1, 32:64] = -Q
+    got = oracle.pack_paired(q, b)
+    rb = oracle.packed_row_bytes(K, b)
+    for n in range(q.shape[0]):
+        want = ex.pack_paired_row_int([int(v) for v in q[n]], b)
+        assert bytes(got[n, : len(want)]) == want
+        assert not got[n, len(want):rb].any()
+
+
+@pytest.mark.parametrize("b", [4, 5, 7, 8, 11, 15])
+def test_unpack_paired_inverts_pack_paired(b):
+    rng = np.random.default_rng(800 + b)
+    Q = oracle.qmax(b)
+    q = rng.integers(-Q, Q + 1, size=(4, 160)).astype(np.int32)
+    assert np.array_equal(oracle.unpack_paired(oracle.pack_paired(q, b), 160, b), q)
+
+
+def test_paired_b8_bytes_are_2x2_transposes():
+    # b = 8: word h of a group holds codes (4h, 4h+2) in its low half and
+    # (4h+1, 4h+3) in its high half, i.e. each block of four int8 codes
+    # [a0, a1, a2, a3] is stored as [a0, a2, a1, a3].
+    rng = np.random.default_rng(81)
+    q = rng.integers(-127, 128, size=(3, 64)).astype(np.int32)
+    p = oracle.pack_paired(q, 8).view(np.int8).astype(np.int32)
+    want = q.reshape(3, 16, 2, 2).transpose(0, 1, 3, 2).reshape(3, 64)
+    assert np.array_equal(p, want)
+
+
+def test_paired_b4_nibble_order():
+    # b = 4: the eight nibbles of word h (low nibble first) are codes
+    # 8h + (0, 2, 4, 6, 1, 3, 5, 7) of the group.
+    rng = np.random.default_rng(41)
+    q = rng.integers(-7, 8, size=(2, 64)).astype(np.int32)
+    p = oracle.pack_paired(q, 4)
+    words = p.view("<u4")
+    for n in range(2):
+        for w in range(8):
+            nib = [(int(words[n, w]) >> (4 * t)) & 15 for t in range(8)]
+            codes = [v - 16 if v >= 8 else v for v in nib]
+            want = [int(q[n, 8 * w + j]) for j in (0, 2, 4, 6, 1, 3, 5, 7)]
+            assert codes == want
+
+
+@pytest.mark.parametrize("b", [5, 6, 9, 13])
+def test_paired_is_a_permutation_of_each_canonical_group(b):
+    # For K a multiple of 32 a canonical group also fills exactly b words, so
+    # the two layouts hold the same multiset of bits word-group by word-group.
+    rng = np.random.default_rng(900 + b)
+    Q = oracle.qmax(b)
+    q = rng.integers(-Q, Q + 1, size=(5, 128)).astype(np.int32)
+    c = np.unpackbits(oracle.pack(q, b), axis=1).reshape(5, -1)
+    p = np.unpackbits(oracle.pack_paired(q, b), axis=1).reshape(5, -1)
+    g_bits = 32 * b
+    for g in range(4):
+        assert np.array_equal(c[:, g * g_bits:(g + 1) * g_bits].sum(1), p[:, g * g_bits:(g + 1) * g_bits].sum(1))
+    assert np.array_equal(oracle.pair_halves(oracle.pack(q, b), 128, b), oracle.pack_paired(q, b))
+
+
+def test_paired_needs_k_multiple_of_32():
+    with pytest.raises(ValueError):
+        oracle.pack_paired(np.zeros((1, 48), np.int32), 5)
+    with pytest.raises(ValueError):
+        oracle.unpack_paired(np.zeros((1, oracle.packed_row_bytes(48, 5)), np.uint8), 48, 5)
