@@ -226,12 +226,14 @@ def time_graph(g, steps, warmup, world=1):
     return max_over_ranks(ms, world)
 
 
-def decode_setup(mpw, W_gpu, b, l2_bytes):
+def decode_setup(mpw, W_gpu, b, l2_bytes, layout="canonical"):
     packed, scales = mpw.quantize_pack(W_gpu, b)
+    if layout != "canonical":
+        packed = mpw.repack(packed, W_gpu.shape[1], b, "canonical", layout)
     return Pool(packed, scales, 4 * l2_bytes)
 
 
-def measure_decode(mpw, pool, b, M, K, N, steps, warmup, world=1, x=None):
+def measure_decode(mpw, pool, b, M, K, N, steps, warmup, world=1, x=None, layout="canonical"):
     import torch
 
     import workloads as wl
@@ -242,7 +244,7 @@ def measure_decode(mpw, pool, b, M, K, N, steps, warmup, world=1, x=None):
 
     def step():
         for i in range(pool.P):
-            mpw.qlinear(x, pool.packed[i], pool.scales[i], b, y=y)
+            mpw.qlinear(x, pool.packed[i], pool.scales[i], b, y=y, layout=layout)
 
     g = graph_of(step)
     ms = time_graph(g, steps, warmup, world)
@@ -281,7 +283,7 @@ def measure_quantize(mpw, W_gpu, b, steps, warmup, l2_bytes):
             "weights_per_s": N * K / (per * 1e-6), "copies": copies}
 
 
-def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup, pool_n):
+def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup, pool_n, layout="canonical"):
     """Same metric through the public call with host buffers: each step copies
     pool_n packed matrices and x host->device, runs the GEMV on each and reads
     y back to the host."""
@@ -299,7 +301,7 @@ def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup
             j = i & 1
             dp[j].copy_(packed_host, non_blocking=True)
             ds[j].copy_(scales_host, non_blocking=True)
-            mpw.qlinear(dx, dp[j], ds[j], b, y=dy)
+            mpw.qlinear(dx, dp[j], ds[j], b, y=dy, layout=layout)
         y_host.copy_(dy, non_blocking=True)
 
     for _ in range(warmup):
@@ -319,7 +321,7 @@ def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup
             "d2h_bytes_per_step": M * N * 2, "ms_per_step": ms / steps}
 
 
-def measure_prefill(mpw, pk, reps=10):
+def measure_prefill(mpw, pk, reps=10, layout="canonical"):
     """Tensor-core prefill GEMM, x 2048x5120 bf16 against the two weight shapes."""
     import torch
 
@@ -332,15 +334,17 @@ def measure_prefill(mpw, pk, reps=10):
         W = wl.gen_weight_torch(N, K, c["sigma"], 11 + N)
         for b in c["bits"]:
             packed, scales = mpw.quantize_pack(W, b)
+            if layout != "canonical":
+                packed = mpw.repack(packed, K, b, "canonical", layout)
             y = torch.empty((c["M"], N), dtype=torch.bfloat16, device="cuda")
             for _ in range(3):
-                mpw.qlinear(x, packed, scales, b, y=y)
+                mpw.qlinear(x, packed, scales, b, y=y, layout=layout)
             torch.cuda.synchronize()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
             for _ in range(reps):
-                mpw.qlinear(x, packed, scales, b, y=y)
+                mpw.qlinear(x, packed, scales, b, y=y, layout=layout)
             e1.record()
             torch.cuda.synchronize()
             us = e0.elapsed_time(e1) * 1e3 / reps
@@ -357,7 +361,7 @@ def measure_prefill(mpw, pk, reps=10):
     return out
 
 
-def measure_recipe(mpw, pk, steps=10, warmup=3):
+def measure_recipe(mpw, pk, steps=10, warmup=3, layout="canonical"):
     """448-matrix mixed-bit decode pass (M = 1) captured in one CUDA graph."""
     import torch
 
@@ -370,7 +374,9 @@ def measure_recipe(mpw, pk, steps=10, warmup=3):
         W = wl.gen_weight_torch(N, K, wl.RECIPE["sigma"], wl.recipe_weight_seed(i))
         packed, scales = mpw.quantize_pack(W, b)
         del W
-        layers.append(mpw.Linear(packed, scales, N, K, b, si, so, nrm))
+        if layout != "canonical":
+            mpw.repack(packed, K, b, "canonical", layout, out=packed)
+        layers.append(mpw.Linear(packed, scales, N, K, b, si, so, nrm, layout=layout))
         wbytes += packed.numel() + scales.numel() * 4
     slots = [torch.zeros((1, wl.SLOT_WIDTH[s]), dtype=torch.bfloat16, device="cuda") for s in range(8)]
     slots[wl.SLOT_H].copy_(wl.gen_x(1, 5120, wl.RECIPE["x_seed"]).cuda())
@@ -473,7 +479,9 @@ def run_case(args):
         layers = []
         for i, ((_, _, N, K), bb, (si, so, nrm)) in enumerate(zip(shapes, bits, links)):
             packed, scales = mpw.quantize_pack(wl.gen_weight_torch(N, K, 0.02, wl.recipe_weight_seed(i)), bb)
-            layers.append(mpw.Linear(packed, scales, N, K, bb, si, so, nrm))
+            if args.layout != "canonical":
+                mpw.repack(packed, K, bb, "canonical", args.layout, out=packed)
+            layers.append(mpw.Linear(packed, scales, N, K, bb, si, so, nrm, layout=args.layout))
         slots = [torch.zeros((1, wl.SLOT_WIDTH[s]), dtype=torch.bfloat16, device="cuda") for s in range(8)]
         for _ in range(args.launches):
             mpw.recipe_run(layers, slots, 1)
@@ -482,9 +490,11 @@ def run_case(args):
             mpw.quantize_pack(W, b)
     else:
         packed, scales = mpw.quantize_pack(W, b)
+        if args.layout != "canonical":
+            packed = mpw.repack(packed, W.shape[1], b, "canonical", args.layout)
         x = wl.gen_x(M, W.shape[1], 1).cuda()
         for _ in range(args.launches):
-            mpw.qlinear(x, packed, scales, b)
+            mpw.qlinear(x, packed, scales, b, layout=args.layout)
     torch.cuda.synchronize()
     return 0
 
@@ -495,7 +505,10 @@ def decode_config(args, pool):
             "N": 4096, "K": 4096, "bits": HEADLINE_BITS, "M": 1,
             "pool_matrices": pool, "l2": "inputs larger than L2: rotating pool of distinct packed "
                                          "matrices totalling > 4x L2 per step",
-            "parallelism": f"replicas x{args.gpus}"}
+            "parallelism": f"replicas x{args.gpus}",
+            "layout": (f"{args.layout}" + (": paired-halves re-ordering of the canonical bits, same bytes, "
+                                           "repacked once outside the timed region"
+                                           if args.layout == "paired" else ""))}
 
 
 # ----------------------------------------------------------------------------
@@ -510,6 +523,8 @@ def main(argv=None):
                     default=None, help="profiling target: run a few launches of one kernel, print nothing")
     ap.add_argument("--bits", type=int, default=HEADLINE_BITS, help="bit width for --case")
     ap.add_argument("--M", type=int, default=1, help="tokens for --case")
+    ap.add_argument("--layout", choices=["canonical", "paired"], default="paired",
+                    help="packed layout the decode and prefill kernels read (repacked outside the timed region)")
     ap.add_argument("--launches", type=int, default=5, help="launches for --case")
     ap.add_argument("--quick", action="store_true",
                     help="headline and e2e only (no sweep, extras or CPU baseline)")
@@ -540,13 +555,14 @@ def main(argv=None):
     W = torch.from_numpy(W_np).cuda()
 
     # ---- headline: b = 6, M = 1 ----
-    pool = decode_setup(mpw, W, HEADLINE_BITS, l2)
+    lay = args.layout
+    pool = decode_setup(mpw, W, HEADLINE_BITS, l2, lay)
     x1 = wl.gen_x(1, K, c["x_seed"]).cuda()
     y1 = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
 
     def step():
         for i in range(pool.P):
-            mpw.qlinear(x1, pool.packed[i], pool.scales[i], HEADLINE_BITS, y=y1)
+            mpw.qlinear(x1, pool.packed[i], pool.scales[i], HEADLINE_BITS, y=y1, layout=lay)
 
     g = graph_of(step)
     with ClockSampler(uuid) as cs:
@@ -565,12 +581,24 @@ def main(argv=None):
     if rank == 0 and not args.quick:
         sweep = []
         for b in DECODE_BITS:
-            p = pool if b == HEADLINE_BITS else decode_setup(mpw, W, b, l2)
+            p = pool if b == HEADLINE_BITS else decode_setup(mpw, W, b, l2, lay)
             for M in DECODE_MS:
-                r = measure_decode(mpw, p, b, M, K, N, max(20, args.steps // 4), 3)
+                r = measure_decode(mpw, p, b, M, K, N, max(20, args.steps // 4), 3, layout=lay)
                 r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
+                r["layout"] = lay
                 sweep.append({k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()
-                              if k in ("b", "M", "us_per_launch", "weight_GBps", "alg_GBps", "pct_hbm")})
+                              if k in ("b", "M", "layout", "us_per_launch", "weight_GBps", "alg_GBps",
+                                       "pct_hbm")})
+            if lay != "canonical":
+                # the canonical rows, read directly (no re-ordering), at M = 1
+                pc = decode_setup(mpw, W, b, l2)
+                r = measure_decode(mpw, pc, b, 1, K, N, max(20, args.steps // 4), 3)
+                r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
+                r["layout"] = "canonical"
+                sweep.append({k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()
+                              if k in ("b", "M", "layout", "us_per_launch", "weight_GBps", "alg_GBps",
+                                       "pct_hbm")})
+                del pc
             if p is not pool:
                 del p
                 torch.cuda.empty_cache()
@@ -584,10 +612,10 @@ def main(argv=None):
         for name, n_, k_ in wl.MLP27B["shapes"][1:]:
             Wm = wl.gen_weight_torch(n_, k_, wl.MLP27B["sigma"], 17 + n_)
             for b in wl.MLP27B["bits"]:
-                pm = decode_setup(mpw, Wm, b, l2)
+                pm = decode_setup(mpw, Wm, b, l2, lay)
                 for M in wl.MLP27B["Ms"]:
                     r = measure_decode(mpw, pm, b, M, k_, n_, 20, 3,
-                                       x=wl.gen_x(M, k_, 1).cuda())
+                                       x=wl.gen_x(M, k_, 1).cuda(), layout=lay)
                     mlp.append({"shape": f"{name} {n_}x{k_}", "b": b, "M": M,
                                 "us_per_launch": round(r["us_per_launch"], 3),
                                 "weight_GBps": round(r["weight_GBps"], 1),
@@ -597,19 +625,20 @@ def main(argv=None):
             del Wm
             torch.cuda.empty_cache()
         extras["mlp27b"] = mlp
-        extras["prefill"] = measure_prefill(mpw, pk)
-        extras["recipe"] = measure_recipe(mpw, pk)
+        extras["prefill"] = measure_prefill(mpw, pk, layout=lay)
+        extras["recipe"] = measure_recipe(mpw, pk, layout=lay)
 
     # ---- e2e: the public call with host buffers ----
     packed_h = pool.packed[0].cpu().pin_memory()
     scales_h = pool.scales[0].cpu().pin_memory()
     x_h = x1.cpu().pin_memory()
     e2e = measure_e2e(mpw, packed_h, scales_h, x_h, HEADLINE_BITS, 1, N, K,
-                      max(3, min(args.steps, 10)), 3, pool.P)
+                      max(3, min(args.steps, 10)), 3, pool.P, layout=lay)
     e2e["value"] = world * e2e["value"]
 
-    traffic = profile_traffic("gemv_tma_decode_b6_m1.json", TMA_GEMV_SOURCES)
-    roof = {"bound": "hbm", "kernel": "gemv_tma_kernel<6>", "achieved": round(achieved, 1),
+    traffic = profile_traffic(f"gemv_tma_decode_b6_m1_{lay}.json", TMA_GEMV_SOURCES)
+    roof = {"bound": "hbm", "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,false,{str(lay == 'paired').lower()}>",
+            "achieved": round(achieved, 1),
             "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
             "traffic": traffic, "alg_bytes_per_launch": alg_bytes,
             "peak_source": pk["source"] + " (copy bandwidth)"}

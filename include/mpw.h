@@ -32,7 +32,11 @@
  *     and returns its status synchronously.  On an argument error nothing is
  *     launched.  No C++ exception crosses this boundary.
  *   - Alignment: `packed` must be 16-byte aligned.  Everything else needs
- *     only its natural alignment.
+ *     only its natural alignment, except where an entry point says otherwise.
+ *   - A second, kernel-private ordering of the same bits ("paired halves",
+ *     mpw_layout below) is read fastest by the decode kernels; mpw_repack
+ *     converts between the two and the *_ex / mpw_linear.layout entry points
+ *     take either.
  */
 #ifndef MPW_H_
 #define MPW_H_
@@ -112,10 +116,11 @@ MPW_API mpw_status mpw_dequantize(const uint8_t* packed, const float* scales,
  *   y        device, bf16 [M, N] row-major; y[m, n] is
  *            bf16_rn(s_n * sum_k x[m, k] * q[n, k]) with an fp32 accumulator.
  *   M >= 1.  M <= 32 runs the decode GEMV kernel (packed rows streamed once,
- *   unpacked in registers); larger M runs the prefill GEMM on tcgen05 tensor
- *   cores with the accumulator in tensor memory.  Codes with b <= 9 are fed
- *   to the tensor cores as exact bf16 values; wider codes are split into
- *   256*hi + lo, both exact in bf16, so no code is ever rounded.
+ *   unpacked in registers, mma.sync tensor cores); larger M runs the prefill
+ *   GEMM on tcgen05 tensor cores with the accumulator in tensor memory.  Every
+ *   code reaches the tensor cores as exact bf16 values: whole when it fits,
+ *   else split into fields (256*hi + lo in the GEMM, 7-bit fields in the
+ *   GEMV), each exact in bf16, so no code is ever rounded.
  * Pages: DynaQuant "Custom kernel architecture" (packed N-bit -> registers ->
  * tensor core; 9-15 bit codes on BF16 tensor cores).
  */
@@ -136,6 +141,41 @@ MPW_API mpw_status mpw_qlinear_path(const uint16_t* x, const uint8_t* packed,
                             int64_t N, int64_t K, uint16_t* y, int path,
                             mpw_stream_t stream);
 
+/* Packed layouts. */
+typedef enum mpw_layout {
+  MPW_LAYOUT_CANONICAL = 0, /* the format above; what mpw_quantize_pack writes */
+  MPW_LAYOUT_PAIRED = 1     /* paired halves; needs K % 32 == 0 */
+} mpw_layout;
+
+/*
+ * mpw_repack -- re-orders packed rows from layout_in to layout_out.
+ *   Paired halves: each row is cut into groups of 32 codes; in group g the
+ *   even codes (32g + 2i, i = 0..15) form one stream and the odd codes
+ *   (32g + 2i + 1) another, code i of a stream in bits [i*b, i*b + b) of it
+ *   (two's complement, LSB first).  Little-endian 32-bit word g*b + h of the
+ *   row holds 16-bit half-word h of the even stream in its low half and
+ *   half-word h of the odd stream in its high half; padding stays zero.  The
+ *   row stride is the canonical one and the layout holds the same bits,
+ *   re-ordered, so a decode kernel can turn the two codes of a pair into one
+ *   bf16x2 operand with a shift and a bit operation.  No page defines this
+ *   layout; it is storage for this library's decode kernels.
+ *   in, out   device, uint8 [N, mpw_packed_row_bytes(K, bits)], 16-B
+ *             aligned; out == in is allowed (in place), other overlap is not.
+ *   layout_in != layout_out, both MPW_LAYOUT_*; K % 32 == 0.
+ */
+MPW_API mpw_status mpw_repack(const uint8_t* in, int64_t N, int64_t K, int bits, int layout_in,
+                              int layout_out, uint8_t* out, mpw_stream_t stream);
+
+/*
+ * mpw_qlinear_ex -- mpw_qlinear_path for packed rows in either layout.
+ *   With MPW_LAYOUT_PAIRED: K % 32 == 0 (else MPW_E_INVALID_ARG) and x
+ *   16-byte aligned (else MPW_E_MISALIGNED).  Results are identical to the
+ *   canonical call on the same codes up to the fp32 summation order.
+ */
+MPW_API mpw_status mpw_qlinear_ex(const uint16_t* x, const uint8_t* packed, const float* scales,
+                                  int bits, int layout, int64_t M, int64_t N, int64_t K,
+                                  uint16_t* y, int path, mpw_stream_t stream);
+
 /*
  * One linear of a recipe stack (DynaQuant "Step 3": every matrix carries its
  * own bit width).  Activations move between caller-owned "slots".
@@ -147,6 +187,9 @@ MPW_API mpw_status mpw_qlinear_path(const uint16_t* x, const uint8_t* packed,
  *             r_m = 1 / sqrt(mean_k x[m, k]^2 + 1e-6), evaluated in fp32 (the
  *             normalisation is a per-token scale of the product; x itself is
  *             not modified).
+ *   layout    MPW_LAYOUT_* of `packed` (paired: K % 32 == 0 and the slots
+ *             16-byte aligned).
+ *   reserved  must be 0.
  */
 typedef struct mpw_linear {
   const uint8_t* packed;
@@ -157,6 +200,8 @@ typedef struct mpw_linear {
   int32_t in_slot;
   int32_t out_slot;
   int32_t norm_input;
+  int32_t layout;
+  int32_t reserved;
 } mpw_linear;
 
 /*

@@ -17,7 +17,8 @@ from dataclasses import dataclass
 
 __all__ = [
     "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
-    "dequantize", "qlinear", "Linear", "recipe_run", "device_error", "status_str",
+    "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str",
+    "LAYOUTS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmpw.so")
@@ -31,6 +32,9 @@ MPW_E_NONFINITE = 5
 MPW_E_TIMEOUT = 6
 
 PATHS = {"auto": 0, "gemv": 1, "gemm": 2}
+# Packed layouts (mpw_layout): the canonical stream and its paired-halves
+# re-ordering, which the decode kernels read fastest (K % 32 == 0).
+LAYOUTS = {"canonical": 0, "paired": 1}
 
 
 class MPWError(RuntimeError):
@@ -49,6 +53,8 @@ class _Linear(ctypes.Structure):
         ("in_slot", ctypes.c_int32),
         ("out_slot", ctypes.c_int32),
         ("norm_input", ctypes.c_int32),
+        ("layout", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
     ]
 
 
@@ -74,6 +80,10 @@ def _load():
     L.mpw_qlinear.restype = c_int
     L.mpw_qlinear_path.argtypes = [vp, vp, vp, c_int, i64, i64, i64, vp, c_int, vp]
     L.mpw_qlinear_path.restype = c_int
+    L.mpw_qlinear_ex.argtypes = [vp, vp, vp, c_int, c_int, i64, i64, i64, vp, c_int, vp]
+    L.mpw_qlinear_ex.restype = c_int
+    L.mpw_repack.argtypes = [vp, i64, i64, c_int, c_int, c_int, vp, vp]
+    L.mpw_repack.restype = c_int
     L.mpw_recipe_run.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp]
     L.mpw_recipe_run.restype = c_int
     L.mpw_device_error.argtypes = [ctypes.POINTER(i32)]
@@ -171,7 +181,26 @@ def dequantize(packed, scales, K: int, bits: int, out=None, stream=None):
     return out
 
 
-def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", stream=None):
+def repack(packed, K: int, bits: int, layout_in: str = "canonical", layout_out: str = "paired", out=None,
+           stream=None):
+    """Re-order packed rows between layouts; ``out=packed`` runs in place."""
+    import torch
+
+    _need(packed, torch.uint8, "packed", 2)
+    if out is None:
+        out = torch.empty_like(packed)
+    _need(out, torch.uint8, "out", 2)
+    if out.shape != packed.shape:
+        raise ValueError("out must have the shape of packed")
+    if packed.shape[1] != packed_row_bytes(K, bits):
+        raise ValueError("packed rows must be exactly packed_row_bytes(K, bits) long")
+    _check(lib.mpw_repack(packed.data_ptr(), packed.shape[0], int(K), int(bits), LAYOUTS[layout_in],
+                          LAYOUTS[layout_out], out.data_ptr(), _stream(stream)), "mpw_repack")
+    return out
+
+
+def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: str = "canonical",
+            stream=None):
     """y = x @ (q * s)^T with x bf16 [M, K]; returns y bf16 [M, N]."""
     import torch
 
@@ -182,13 +211,13 @@ def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", stream=Non
     N = packed.shape[0]
     if scales.shape[0] != N:
         raise ValueError("scales must have one entry per packed row")
-    if packed.shape[1] < packed_row_bytes(K, bits):
-        raise ValueError("packed rows are shorter than packed_row_bytes(K, bits)")
+    if packed.shape[1] != packed_row_bytes(K, bits):
+        raise ValueError("packed rows must be exactly packed_row_bytes(K, bits) long")
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(y, torch.bfloat16, "y")
-    _check(lib.mpw_qlinear_path(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits), M, N, K,
-                                y.data_ptr(), PATHS[path], _stream(stream)), "mpw_qlinear")
+    _check(lib.mpw_qlinear_ex(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits), LAYOUTS[layout],
+                              M, N, K, y.data_ptr(), PATHS[path], _stream(stream)), "mpw_qlinear")
     return y
 
 
@@ -203,6 +232,7 @@ class Linear:
     in_slot: int
     out_slot: int
     norm_input: bool = False
+    layout: str = "canonical"
 
 
 def recipe_run(layers, slots, M: int, stream=None):
@@ -210,7 +240,7 @@ def recipe_run(layers, slots, M: int, stream=None):
     arr = (_Linear * len(layers))()
     for i, L in enumerate(layers):
         arr[i] = _Linear(L.packed.data_ptr(), L.scales.data_ptr(), int(L.N), int(L.K), int(L.bits),
-                         int(L.in_slot), int(L.out_slot), int(bool(L.norm_input)))
+                         int(L.in_slot), int(L.out_slot), int(bool(L.norm_input)), LAYOUTS[L.layout], 0)
     ptrs = (ctypes.c_void_p * len(slots))(*[s.data_ptr() for s in slots])
     _check(lib.mpw_recipe_run(arr, len(layers), ptrs, len(slots), int(M), _stream(stream)),
            "mpw_recipe_run")

@@ -10,6 +10,9 @@
 
 namespace mpw {
 
+static_assert(MPW_LAYOUT_CANONICAL == kLayoutCanonical && MPW_LAYOUT_PAIRED == kLayoutPaired,
+              "layout values of the C ABI and the kernels agree");
+
 // Device-side error word: set by bounded waits that give up.
 __device__ int32_t g_device_error = 0;
 
@@ -32,6 +35,8 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 mpw_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MPW_OK : MPW_E_CUDA; }
 
 bool bits_ok(int bits) { return bits >= kMinBits && bits <= kMaxBits; }
+
+bool layout_ok(int layout) { return layout == MPW_LAYOUT_CANONICAL || layout == MPW_LAYOUT_PAIRED; }
 
 }  // namespace
 
@@ -106,7 +111,7 @@ const char* mpw_status_str(int status) {
   }
 }
 
-int mpw_version(void) { return 100; }
+int mpw_version(void) { return 200; }
 
 size_t mpw_packed_row_bytes(int64_t K, int bits) {
   if (!bits_ok(bits) || K < 1) return 0;
@@ -145,29 +150,53 @@ mpw_status mpw_dequantize(const uint8_t* packed, const float* scales, int64_t N,
       launch_dequantize(packed, scales, N, K, bits, W_hat, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-mpw_status mpw_qlinear_path(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
-                            int64_t M, int64_t N, int64_t K, uint16_t* y, int path,
-                            mpw_stream_t stream) {
+mpw_status mpw_repack(const uint8_t* in, int64_t N, int64_t K, int bits, int layout_in, int layout_out,
+                      uint8_t* out, mpw_stream_t stream) {
+  if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
+  if (in == nullptr || out == nullptr || N < 1 || K < 1 || K > 0x3fffffff || K % 32 != 0)
+    return MPW_E_INVALID_ARG;
+  if (!layout_ok(layout_in) || !layout_ok(layout_out) || layout_in == layout_out) return MPW_E_INVALID_ARG;
+  if (!aligned(in, 16) || !aligned(out, 16)) return MPW_E_MISALIGNED;
+  if (in != out) {
+    // the kernel may run in place, but not on partly overlapping rows
+    const size_t bytes = static_cast<size_t>(N) * mpw_packed_row_bytes(K, bits);
+    const uintptr_t a = reinterpret_cast<uintptr_t>(in), b = reinterpret_cast<uintptr_t>(out);
+    if (a < b + bytes && b < a + bytes) return MPW_E_INVALID_ARG;
+  }
+  return from_cuda(launch_repack(in, N, K, bits, out, layout_out == MPW_LAYOUT_PAIRED,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mpw_status mpw_qlinear_ex(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
+                          int64_t M, int64_t N, int64_t K, uint16_t* y, int path, mpw_stream_t stream) {
   if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
   if (x == nullptr || packed == nullptr || scales == nullptr || y == nullptr || M < 1 || N < 1 ||
       K < 1)
     return MPW_E_INVALID_ARG;
   if (N > 0x7fffffff || K > 0x3fffffff || M > 0x7fffffff) return MPW_E_INVALID_ARG;
-  if (path < MPW_PATH_AUTO || path > MPW_PATH_GEMM) return MPW_E_INVALID_ARG;
-  if (!aligned(packed, 16) || !aligned(x, 2) || !aligned(y, 2) || !aligned(scales, 4))
+  if (path < MPW_PATH_AUTO || path > MPW_PATH_GEMM || !layout_ok(layout)) return MPW_E_INVALID_ARG;
+  const bool paired = layout == MPW_LAYOUT_PAIRED;
+  if (paired && K % 32 != 0) return MPW_E_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(x, paired ? 16 : 2) || !aligned(y, 2) || !aligned(scales, 4))
     return MPW_E_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool want_gemm = path == MPW_PATH_GEMM || (path == MPW_PATH_AUTO && M > 32);
   if (want_gemm && gemm_supported(M, N, K) && aligned(x, 16)) {
-    return from_cuda(launch_gemm(x, packed, scales, bits, M, N, K, y, device_error_word(), s));
+    return from_cuda(launch_gemm(x, packed, scales, bits, layout, M, N, K, y, device_error_word(), s));
   }
   if (path == MPW_PATH_GEMM) return MPW_E_INVALID_ARG;  // shape the GEMM does not take
-  return from_cuda(launch_gemv(x, packed, scales, bits, M, N, K, y, false, s));
+  return from_cuda(launch_gemv(x, packed, scales, bits, layout, M, N, K, y, false, s));
+}
+
+mpw_status mpw_qlinear_path(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                            int64_t M, int64_t N, int64_t K, uint16_t* y, int path,
+                            mpw_stream_t stream) {
+  return mpw_qlinear_ex(x, packed, scales, bits, MPW_LAYOUT_CANONICAL, M, N, K, y, path, stream);
 }
 
 mpw_status mpw_qlinear(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
                        int64_t M, int64_t N, int64_t K, uint16_t* y, mpw_stream_t stream) {
-  return mpw_qlinear_path(x, packed, scales, bits, M, N, K, y, MPW_PATH_AUTO, stream);
+  return mpw_qlinear_ex(x, packed, scales, bits, MPW_LAYOUT_CANONICAL, M, N, K, y, MPW_PATH_AUTO, stream);
 }
 
 mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count, uint16_t* const* slots,
@@ -183,13 +212,16 @@ mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count, uint16_t* con
     if (L.in_slot < 0 || L.in_slot >= num_slots || L.out_slot < 0 || L.out_slot >= num_slots ||
         L.in_slot == L.out_slot)
       return MPW_E_INVALID_ARG;
+    if (!layout_ok(L.layout) || L.reserved != 0) return MPW_E_INVALID_ARG;
+    if (L.layout == MPW_LAYOUT_PAIRED && L.K % 32 != 0) return MPW_E_INVALID_ARG;
     if (slots[L.in_slot] == nullptr || slots[L.out_slot] == nullptr) return MPW_E_INVALID_ARG;
     if (!aligned(L.packed, 16) || !aligned(L.scales, 4)) return MPW_E_MISALIGNED;
+    if (L.layout == MPW_LAYOUT_PAIRED && !aligned(slots[L.in_slot], 16)) return MPW_E_MISALIGNED;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   for (int64_t i = 0; i < count; ++i) {
     const mpw_linear& L = layers[i];
-    cudaError_t e = launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, M, L.N, L.K,
+    cudaError_t e = launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, L.layout, M, L.N, L.K,
                                 slots[L.out_slot], L.norm_input != 0, s);
     if (e != cudaSuccess) return MPW_E_CUDA;
   }

@@ -20,6 +20,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace mpw {
 namespace dec {
 
@@ -169,6 +171,72 @@ __device__ __forceinline__ void permute_x(uint32_t (&xw)[16]) {
 #pragma unroll
     for (int p = 0; p < 16; ++p) xw[p] = o[p];
   }
+}
+
+// ---------------------------------------------------------------------------
+// Paired-halves layout (a re-ordering of the canonical bits, K % 32 == 0):
+// word h of a group holds half-word h of the stream of its even codes in the
+// low 16 bits and half-word h of the stream of its odd codes in the high 16
+// bits; code i of a stream occupies bits [i*B, i*B+B) of that stream.  The
+// two codes of pair i = (2i, 2i+1) therefore sit at the same offset in the
+// two halves of one word -- or, when the field crosses a half-word boundary,
+// of two consecutive words -- so a shift and one LOP3 (two of each when the
+// field crosses) give their bf16x2 pair, already in the k order of the raw x
+// pairs (x[2i], x[2i+1]): no x permutation.
+// ---------------------------------------------------------------------------
+
+// Field [F0, F0+NB) of both codes of pair I as bf16 values 128 + field, the
+// top bit of the field flipped when SIGNED (two's complement -> offset binary).
+template <int B, int I, int F0, int NB, bool SIGNED>
+__device__ __forceinline__ uint32_t paired_field(const uint32_t (&w)[B + 1]) {
+  constexpr int o = I * B + F0;
+  constexpr int h = o >> 4, r = o & 15;
+  constexpr uint32_t fm = ((1u << NB) - 1u) * 0x10001u;
+  constexpr uint32_t xm = 0x43004300u | (SIGNED ? (1u << (NB - 1)) * 0x10001u : 0u);
+  uint32_t t;
+  if constexpr (r + NB <= 16) {
+    t = r == 0 ? w[h] : (w[h] >> r);
+  } else {
+    // low part from word h, high part from word h+1, in both halves at once
+    constexpr uint32_t sel = ((1u << (16 - r)) - 1u) * 0x10001u;
+    t = ((w[h] >> r) & sel) | ((w[h + 1] << (16 - r)) & ~sel);
+  }
+  return and_xor(t, fm, xm);
+}
+
+template <int B, int I>
+__device__ __forceinline__ void paired_pair(const uint32_t (&w)[B + 1], uint32_t (&v)[Exp<B>::parts][16]) {
+  const uint32_t one = pair_of(1);
+  if constexpr (B <= 7) {
+    v[0][I] = bf2_fma(paired_field<B, I, 0, B, true>(w), one, pair_of(-(128 + (1 << (B - 1)))));
+  } else if constexpr (B == 8) {
+    // q = lo + 16 * hi: low nibble unsigned, high nibble signed
+    v[0][I] = bf2_fma(paired_field<B, I, 0, 4, false>(w), one, pair_of(-128));
+    v[1][I] = bf2_fma(paired_field<B, I, 4, 4, true>(w), pair_of(16), pair_of(-16 * 136));
+  } else if constexpr (B <= 14) {
+    // q = lo7 + 128 * hi with hi = the signed top B-7 bits
+    v[0][I] = bf2_fma(paired_field<B, I, 0, 7, false>(w), one, pair_of(-128));
+    v[1][I] = bf2_fma(paired_field<B, I, 7, B - 7, true>(w), pair_of(128),
+                      pair_of(-128 * (128 + (1 << (B - 8)))));
+  } else {
+    // q = lo7 + 128 * mid7 + 16384 * (top' - 1), top' = flipped sign bit
+    v[0][I] = bf2_fma(paired_field<B, I, 0, 7, false>(w), one, pair_of(-128));
+    v[1][I] = bf2_fma(paired_field<B, I, 7, 7, false>(w), pair_of(128), pair_of(-128 * 128));
+    v[2][I] = bf2_fma(paired_field<B, I, 14, 1, true>(w), pair_of(16384), pair_of(-16384 * 129));
+  }
+}
+
+template <int B, int... I>
+__device__ __forceinline__ void paired_all(const uint32_t (&w)[B + 1], uint32_t (&v)[Exp<B>::parts][16],
+                                           std::integer_sequence<int, I...>) {
+  (paired_pair<B, I>(w, v), ...);
+}
+
+// Expands one 32-code group of a paired-halves row; v[part][i] holds pair i
+// = (code 2i, code 2i+1), the k order of the raw x pairs.
+template <int B>
+__device__ __forceinline__ void expand_paired(const uint32_t (&w)[B + 1], uint32_t (&v)[Exp<B>::parts][16]) {
+  paired_all<B>(w, v, std::make_integer_sequence<int, 16>{});
 }
 
 __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

@@ -67,6 +67,26 @@ __device__ __forceinline__ float code_f32(const uint32_t (&w)[B + 1], int j) {
   return __uint_as_float((t & kMask) ^ kMagic) - kOffset;
 }
 
+// Code j (0..31) of a 32-code group of a paired-halves row: even codes form
+// the stream in the low half-words, odd codes the stream in the high ones.
+template <int B>
+__device__ __forceinline__ float code_f32_paired(const uint32_t (&w)[B + 1], int j) {
+  const int o = (j >> 1) * B;
+  const int h = o >> 4, r = o & 15;
+  // half-words h and h+1 of the code's stream as one 32-bit window
+  const uint32_t win = __byte_perm(w[h], w[h + 1], (j & 1) ? 0x7632 : 0x5410);
+  constexpr uint32_t kMask = (1u << B) - 1u;
+  constexpr uint32_t kMagic = 0x4B000000u | (1u << (B - 1));
+  constexpr float kOffset = 8388608.0f + static_cast<float>(1 << (B - 1));
+  return __uint_as_float(((win >> r) & kMask) ^ kMagic) - kOffset;
+}
+
+template <int B, bool PAIRED>
+__device__ __forceinline__ float code_at(const uint32_t (&w)[B + 1], int j) {
+  if constexpr (PAIRED) return code_f32_paired<B>(w, j);
+  else return code_f32<B>(w, j);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -84,7 +104,7 @@ __device__ __forceinline__ void load_group(const uint32_t* __restrict__ rowp, in
   w[B] = 0u;
 }
 
-template <int B>
+template <int B, bool PAIRED>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ packed,
             const float* __restrict__ scales, uint16_t* __restrict__ y, int M, int N, int K, int rw,
@@ -191,7 +211,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restric
       if (C::HL) {
 #pragma unroll
         for (int p = 0; p < 16; ++p) {
-          const float q0 = code_f32<B>(wcur, 2 * p), q1 = code_f32<B>(wcur, 2 * p + 1);
+          const float q0 = code_at<B, PAIRED>(wcur, 2 * p), q1 = code_at<B, PAIRED>(wcur, 2 * p + 1);
           const int i0 = static_cast<int>(q0), i1 = static_cast<int>(q1);
           const float l0 = static_cast<float>(i0 & 255), l1 = static_cast<float>(i1 & 255);
           va[p] = pack_bf16x2(q0 - l0, q1 - l1);   // 256 * hi, exact
@@ -199,7 +219,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restric
         }
       } else {
 #pragma unroll
-        for (int p = 0; p < 16; ++p) va[p] = pack_bf16x2(code_f32<B>(wcur, 2 * p), code_f32<B>(wcur, 2 * p + 1));
+        for (int p = 0; p < 16; ++p) va[p] = pack_bf16x2(code_at<B, PAIRED>(wcur, 2 * p), code_at<B, PAIRED>(wcur, 2 * p + 1));
       }
       ok = ptx::mbar_wait(empty_a(s), ((kb / SA) & 1) ^ 1, err);
       if (!ok) break;
@@ -244,7 +264,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restric
   }
 }
 
-template <int B>
+template <int B, bool PAIRED>
 cudaError_t run_gemm(const uint16_t* x, const uint8_t* packed, const float* scales, int64_t M,
                      int64_t N, int64_t K, uint16_t* y, int32_t* err, cudaStream_t stream) {
   auto encode = tensor_map_encoder();
@@ -258,7 +278,7 @@ cudaError_t run_gemm(const uint16_t* x, const uint8_t* packed, const float* scal
                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = gemm_kernel<B>;
+  auto kern = gemm_kernel<B, PAIRED>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kSmemBytes);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>((N + BM - 1) / BM), static_cast<unsigned>((M + BN - 1) / BN));
@@ -275,24 +295,31 @@ bool gemm_supported(int64_t M, int64_t N, int64_t K) {
   return K % 8 == 0 && M >= 1 && N >= 1 && (M + BN - 1) / BN <= 65535;
 }
 
-cudaError_t launch_gemm(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
-                        int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* err,
-                        cudaStream_t stream) {
+template <bool PAIRED>
+cudaError_t gemm_layout(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int64_t M,
+                        int64_t N, int64_t K, uint16_t* y, int32_t* err, cudaStream_t stream) {
   switch (bits) {
-    case 4: return run_gemm<4>(x, packed, scales, M, N, K, y, err, stream);
-    case 5: return run_gemm<5>(x, packed, scales, M, N, K, y, err, stream);
-    case 6: return run_gemm<6>(x, packed, scales, M, N, K, y, err, stream);
-    case 7: return run_gemm<7>(x, packed, scales, M, N, K, y, err, stream);
-    case 8: return run_gemm<8>(x, packed, scales, M, N, K, y, err, stream);
-    case 9: return run_gemm<9>(x, packed, scales, M, N, K, y, err, stream);
-    case 10: return run_gemm<10>(x, packed, scales, M, N, K, y, err, stream);
-    case 11: return run_gemm<11>(x, packed, scales, M, N, K, y, err, stream);
-    case 12: return run_gemm<12>(x, packed, scales, M, N, K, y, err, stream);
-    case 13: return run_gemm<13>(x, packed, scales, M, N, K, y, err, stream);
-    case 14: return run_gemm<14>(x, packed, scales, M, N, K, y, err, stream);
-    case 15: return run_gemm<15>(x, packed, scales, M, N, K, y, err, stream);
+    case 4: return run_gemm<4, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 5: return run_gemm<5, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 6: return run_gemm<6, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 7: return run_gemm<7, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 8: return run_gemm<8, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 9: return run_gemm<9, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 10: return run_gemm<10, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 11: return run_gemm<11, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 12: return run_gemm<12, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 13: return run_gemm<13, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 14: return run_gemm<14, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 15: return run_gemm<15, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_gemm(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
+                        int64_t M, int64_t N, int64_t K, uint16_t* y, int32_t* err,
+                        cudaStream_t stream) {
+  if (layout == kLayoutPaired) return gemm_layout<true>(x, packed, scales, bits, M, N, K, y, err, stream);
+  return gemm_layout<false>(x, packed, scales, bits, M, N, K, y, err, stream);
 }
 
 }  // namespace mpw

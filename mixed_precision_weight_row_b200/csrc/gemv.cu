@@ -440,22 +440,25 @@ cudaError_t gemv_bits(const uint16_t* x, int64_t M, const uint8_t* packed, const
 }  // namespace
 
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
-                        int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm_input,
+                        int layout, int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm_input,
                         cudaStream_t stream) {
-  // Tensor-core decode kernel in passes of up to 32 tokens (8 with norm_input).
-  // MPW_GEMV_KERNEL=mma selects the register-streaming variant (tuning aid).
+  // Tensor-core decode kernels in passes of up to 32 tokens (8 with
+  // norm_input).  MPW_GEMV_KERNEL=mma selects the register-streaming variant
+  // for canonical rows (tuning aid).
   static const bool use_mma = [] {
     const char* e = getenv("MPW_GEMV_KERNEL");
     return e != nullptr && e[0] == 'm';
   }();
   const int64_t pass = norm_input ? 8 : 32;
   const int64_t m1 = M < pass ? M : pass;
-  const bool tma = !use_mma && gemv_tma_supported(m1, N, K, norm_input);
+  const bool paired = layout == kLayoutPaired;
+  const bool tma = (paired || !use_mma) && gemv_tma_supported(x, m1, N, K, norm_input);
+  if (paired && !tma) return cudaErrorInvalidValue;
   if (tma || gemv_mma_supported(m1, N, K, norm_input)) {
     for (int64_t m0 = 0; m0 < M; m0 += pass) {
       const int64_t mt = M - m0 < pass ? M - m0 : pass;
-      cudaError_t e = tma ? launch_gemv_tma(x + m0 * K, packed, scales, bits, mt, N, K, y + m0 * N, norm_input,
-                                            /*pdl=*/true, stream)
+      cudaError_t e = tma ? launch_gemv_tma(x + m0 * K, packed, scales, bits, layout, mt, N, K, y + m0 * N,
+                                            norm_input, /*pdl=*/true, stream)
                           : launch_gemv_mma(x + m0 * K, packed, scales, bits, mt, N, K, y + m0 * N, norm_input,
                                             /*pdl=*/true, stream);
       if (e != cudaSuccess) return e;

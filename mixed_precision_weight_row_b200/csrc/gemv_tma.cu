@@ -1,5 +1,6 @@
-// Decode linear for M <= 32 tokens: packed weights streamed by TMA into a
-// shared-memory ring, expanded in registers, multiplied on tensor cores.
+// Decode linear for M <= 32 tokens: packed weights and x streamed by TMA into
+// a shared-memory ring, weights expanded in registers, multiplied on tensor
+// cores.
 //   y[m, n] = bf16(s_n * sum_k x[m, k] * q[n, k])
 //
 // DynaQuant, "Custom kernel architecture": packed N-bit weights are read from
@@ -7,26 +8,26 @@
 // in decode the bytes saved are the speedup (the layer is bandwidth-bound:
 // quantization tutorial, closing note).
 //
-// A CTA owns a 16-row tile of W (one cluster of 1..8 CTAs splits the tile's K
-// range).  Warp 4 is the producer: one lane walks the CTA's chunks (128 codes
-// = 16*B bytes per row) and issues one 2D TMA per chunk, {16*B bytes x 16
-// rows}, into a ring of S stages of four chunks each (mbarrier completion,
-// rows past N and bytes past the row read as zeros).  Warps 0..3 consume: warp
-// w takes chunk 4s+w of stage s, reads the 32-code group of lane tig for rows
-// g and g+8 from shared memory (B words per row), expands it to exact bf16
-// (expand.cuh) and issues mma.sync m16n8k16 against its x fragment (token g,
-// read through L1).  The stage is released to the producer as soon as its
-// words are in registers, so the memory system always has S stages of the
-// tile in flight independent of how many loads the warps themselves could
-// keep outstanding.  Partial sums of the K slices are reduced through shared
+// A CTA owns a 16-row tile of W (a cluster of 1..8 CTAs splits the tile's K
+// range).  The last warp is the producer: one lane walks the CTA's 128-code
+// chunks and, per chunk, issues one 2D TMA of the packed rows ({16*B bytes x
+// 16 rows}) and one of x ({128 values x M tokens}) into a ring of stages of
+// kCW*kCH chunks each (mbarrier completion; rows past N, bytes past the row
+// and values past K read as zeros).  Consumer warp w takes kCH consecutive
+// chunks of each stage: per chunk, the 32-code group of lane tig for rows g
+// and g+8 (B words per row) and its x fragment for token g, both from shared
+// memory; it expands the codes to exact bf16 (expand.cuh; canonical or
+// paired-halves layout) and issues mma.sync m16n8k16 into two alternating
+// fp32 accumulators, releasing the stage once its last words are read.  Partial sums of the K slices are reduced through shared
 // memory and distributed shared memory into the cluster's first CTA, which
 // applies the row scale (and the rms scale with norm_input) and writes bf16.
 //
 // Programmatic dependent launch: every thread lets the next kernel launch at
-// once; the producer's TMA loads read only W and never wait, the consumers
-// wait (griddepcontrol.wait) before touching x or y.  In a chain of linears
-// the next layer's weights stream in while the previous kernel drains.  Every mbarrier wait is bounded (2 s), after which
-// the kernel records an error in the device error word and winds down.
+// once.  The producer issues the weight loads of the first stages before
+// griddepcontrol.wait and the x loads after it; the thread that writes y
+// waits too.  In a chain of linears the next layer's weights stream in while
+// the previous kernel drains.  Every mbarrier wait is bounded (2 s), after
+// which the kernel records an error in the device error word and winds down.
 #include <cooperative_groups.h>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -47,18 +48,30 @@ namespace {
 
 using namespace dec;
 
-constexpr int kCW = 4;                 // consumer warps
+constexpr int kCW = 4;                  // consumer warps
+constexpr int kCH = 2;                  // chunks per consumer warp and stage
+constexpr int kSC = kCW * kCH;          // chunks per stage
 constexpr int kThreads = (kCW + 1) * 32;
-constexpr int kChunk = 128;            // codes per chunk
+constexpr int kChunk = 128;             // codes per chunk and row
 constexpr int kNormMaxM = 8;
+constexpr int kMaxStages = 8;
+constexpr uint32_t kRingBudget = 48u * 1024u;
 
-// Read-only zeros for lanes without a token (past M).
-__device__ __align__(16) uint32_t g_tma_zero_page[16];
+// Bytes of one stage: kSC weight chunks (16 rows x 16*B bytes) followed by
+// kSC x chunks (M tokens x 128 bf16).
+__host__ __device__ constexpr uint32_t stage_bytes(int B, int M) {
+  return static_cast<uint32_t>(kSC) * 256u * static_cast<uint32_t>(B + M);
+}
 
-template <int B>
-constexpr int ring_stages() {
-  // one stage = 4 chunks x 16 rows x 16*B bytes = 1 KB * B
-  return B <= 6 ? 6 : (B <= 10 ? 4 : 3);
+int ring_stages(int B, int M) {
+  // MPW_GEMV_RING_KB overrides the ring budget (tuning aid)
+  static const uint32_t budget = [] {
+    const char* e = getenv("MPW_GEMV_RING_KB");
+    const int v = e ? atoi(e) : 0;
+    return v >= 8 && v <= 192 ? static_cast<uint32_t>(v) * 1024u : kRingBudget;
+  }();
+  const int s = static_cast<int>(budget / stage_bytes(B, M));
+  return s < 2 ? 2 : (s > kMaxStages ? kMaxStages : s);
 }
 
 template <int B>
@@ -82,24 +95,33 @@ __device__ __forceinline__ void lds_words(const uint8_t* p, uint32_t (&w)[B + 1]
   w[B] = 0u;
 }
 
-template <int B, int NT, bool NORM>
-__global__ void __launch_bounds__(kThreads)
-gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t* __restrict__ x, int M,
-                const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int32_t* err) {
+// CTAs per SM the register budget is sized for: wide codes and many tokens
+// need more registers per thread (spill-free), narrow ones leave room for
+// four CTAs.
+template <int B, int NT>
+constexpr int min_ctas() {
+  return NT == 1 ? (B <= 7 ? 4 : 3) : (NT == 2 ? 2 : 1);
+}
+
+template <int B, int NT, bool NORM, bool PAIRED>
+__global__ void __launch_bounds__(kThreads, min_ctas<B, NT>())
+gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                int M, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
+                int32_t* err) {
   constexpr int P = Exp<B>::parts;
   constexpr int NS = NORM ? kNormMaxM : 1;
-  constexpr int S = ring_stages<B>();
-  constexpr uint32_t kChunkBytes = 16u * 16u * B;   // 16 rows x 16*B bytes
-  constexpr uint32_t kStageBytes = 4u * kChunkBytes;
+  constexpr uint32_t kWChunk = 256u * B;        // 16 rows x 16*B bytes
+  const uint32_t x_chunk = 256u * M;            // M tokens x 128 bf16
+  const uint32_t w_part = kSC * kWChunk;
+  const uint32_t st_bytes = stage_bytes(B, M);
   extern __shared__ __align__(128) uint8_t tsmem[];
-  __shared__ __align__(8) uint64_t bars[2 * S];
+  __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
   __shared__ float red[kCW][NT][32][4];
   __shared__ float cl_red[8][NT][32][4];
   __shared__ float ss_red[kCW][NS];
   __shared__ float cl_ss[8][NS];
+  __shared__ __align__(16) uint4 zero_x[4];   // x fragment of lanes without a token
 
-  // The next kernel in the stream may launch right away: it only streams its
-  // own weights until its consumers pass griddepcontrol.wait.
   asm volatile("griddepcontrol.launch_dependents;");
   cg::cluster_group cluster = cg::this_cluster();
   const int KC = static_cast<int>(cluster.num_blocks());
@@ -111,12 +133,12 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t* __re
   const int cpc = (chunks + KC - 1) / KC;
   const int cb = cr * cpc;
   const int ce = min(chunks, cb + cpc);
-  const int n_stages = ce > cb ? (ce - cb + 3) / 4 : 0;
+  const int n_stages = ce > cb ? (ce - cb + kSC - 1) / kSC : 0;
   const int r0 = tile * 16;
   const uint32_t base = ptx::smem_addr(tsmem);
   const uint32_t bar0 = ptx::smem_addr(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
-  auto empty = [&](int s) { return bar0 + 8u * (S + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (kMaxStages + s); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -125,119 +147,148 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t* __re
     }
     ptx::mbar_fence_init();
   }
+  if (threadIdx.x < 4) zero_x[threadIdx.x] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
 
   if (warp == kCW) {
     // ---------------- producer ----------------
     if (lane == 0) {
       ptx::prefetch_tmap(&tmap_w);
-      int issued = 0;
-      for (int s = 0; s < n_stages; ++s) {
-        const int slot = s % S;
-        if (!ptx::mbar_wait(empty(slot), ((s / S) & 1) ^ 1, err)) break;
-        const int c_first = cb + 4 * s;
-        const int nvalid = min(4, ce - c_first);
-        ptx::mbar_arrive_expect_tx(full(slot), nvalid * kChunkBytes);
-        for (int j = 0; j < nvalid; ++j)
-          ptx::tma_load_2d(base + slot * kStageBytes + j * kChunkBytes, &tmap_w, full(slot),
-                           (c_first + j) * 16 * B, r0);
+      ptx::prefetch_tmap(&tmap_x);
+      auto nvalid = [&](int s) { return min(kSC, ce - (cb + kSC * s)); };
+      auto issue_w = [&](int s, int slot) {
+        const int c0 = cb + kSC * s, nv = nvalid(s);
+        ptx::mbar_arrive_expect_tx(full(slot), nv * (kWChunk + x_chunk));
+        for (int j = 0; j < nv; ++j)
+          ptx::tma_load_2d(base + slot * st_bytes + j * kWChunk, &tmap_w, full(slot), (c0 + j) * 16 * B, r0);
+      };
+      auto issue_x = [&](int s, int slot) {
+        const int c0 = cb + kSC * s, nv = nvalid(s);
+        for (int j = 0; j < nv; ++j)
+          ptx::tma_load_2d(base + slot * st_bytes + w_part + j * x_chunk, &tmap_x, full(slot),
+                           (c0 + j) * kChunk, 0);
+      };
+      const int pre = min(S, n_stages);
+      // weights do not depend on the previous kernel in the stream; x does
+      for (int s = 0; s < pre; ++s) issue_w(s, s);
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      for (int s = 0; s < pre; ++s) issue_x(s, s);
+      int issued = pre;
+      int slot = 0;
+      uint32_t phase = 0;   // phase of empty(slot) that frees it for stage s
+      for (int s = pre; s < n_stages; ++s) {
+        if (!ptx::mbar_wait(empty(slot), phase, err)) break;
+        issue_w(s, slot);
+        issue_x(s, slot);
         issued = s + 1;
+        if (++slot == S) {
+          slot = 0;
+          phase ^= 1u;
+        }
       }
       // nothing may still be landing in shared memory when the CTA exits
       for (int s = max(0, issued - S); s < issued; ++s) ptx::mbar_wait(full(s % S), (s / S) & 1, err);
     }
   } else {
     // ---------------- consumers ----------------
-    // x (and y) may belong to the previous kernel in the stream
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    float acc[NT][4];
+    float acc[2][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) acc[a][nt][0] = acc[a][nt][1] = acc[a][nt][2] = acc[a][nt][3] = 0.0f;
     float ss[NS];
 #pragma unroll
     for (int t = 0; t < NS; ++t) ss[t] = 0.0f;
 
-    const bool xvec = (K % 8) == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0;
-    const uint16_t* zero_x = reinterpret_cast<const uint16_t*>(g_tma_zero_page);
-    for (int s = 0; s < n_stages; ++s) {
-      const int slot = s % S;
-      const int c = cb + 4 * s + warp;
-      const bool active = c < ce;
-      // x fragments of this chunk (independent of the ring: issued first)
+    // lanes without a token read a zero area (an address select, not a value
+    // select per register)
+    uint32_t x_lane[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) x_lane[nt] = (g + 8 * nt) * 256 + tig * 64;
+    const uint32_t w_lane = tig * 4 * B + g * 16 * B;
+
+    // One chunk: B words of rows g and g+8, the x fragment of token g, expand,
+    // (release the stage after its last chunk), MMAs.
+    auto chunk = [&](const uint8_t* st, int jc, bool active, bool release, uint32_t rel_bar) {
+      uint32_t wa[B + 1], wb[B + 1];
+      const uint8_t* wr = st + jc * kWChunk + w_lane;
+      lds_words<B>(wr, wa);
+      lds_words<B>(wr + 8 * 16 * B, wb);
+      const uint8_t* xc = st + w_part + jc * x_chunk;
       uint32_t xw[NT][16];
-      const int grp = 4 * c + tig;
-      const int k0 = grp * 32;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const int tok = g + 8 * nt;
-        const bool on = active && tok < M;
-        if (xvec && k0 + 32 <= K) {
-          const uint4* p = reinterpret_cast<const uint4*>(on ? x + static_cast<size_t>(tok) * K + k0 : zero_x);
+        const uint4* px = g + 8 * nt < M ? reinterpret_cast<const uint4*>(xc + x_lane[nt]) : zero_x;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 v = __ldg(p + q);
-            xw[nt][4 * q] = v.x; xw[nt][4 * q + 1] = v.y; xw[nt][4 * q + 2] = v.z; xw[nt][4 * q + 3] = v.w;
-          }
-        } else {
-          const uint16_t* xr = x + static_cast<size_t>(tok < M ? tok : 0) * K;
-#pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const int k = k0 + 2 * m;
-            const uint32_t lo = (on && k < K) ? __ldg(xr + k) : 0u;
-            const uint32_t hi = (on && k + 1 < K) ? __ldg(xr + k + 1) : 0u;
-            xw[nt][m] = lo | (hi << 16);
-          }
+        for (int q = 0; q < 4; ++q) {
+          const uint4 v = px[q];
+          xw[nt][4 * q] = v.x; xw[nt][4 * q + 1] = v.y; xw[nt][4 * q + 2] = v.z; xw[nt][4 * q + 3] = v.w;
         }
       }
       if (NORM && active) {
         // squares of x for the rms scale: 4 of the chunk's 128 values per lane
-        const int kk = c * kChunk + 4 * lane;
 #pragma unroll
         for (int t = 0; t < NS; ++t) {
           if (t < M) {
-            const uint16_t* xr = x + static_cast<size_t>(t) * K;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              if (kk + e < K) {
-                const float v = __uint_as_float(static_cast<uint32_t>(__ldg(xr + kk + e)) << 16);
-                ss[t] = fmaf(v, v, ss[t]);
-              }
-            }
+            const uint2 v = *reinterpret_cast<const uint2*>(xc + t * 256 + lane * 8);
+            const float a0 = __uint_as_float(v.x << 16), a1 = __uint_as_float(v.x & 0xFFFF0000u);
+            const float a2 = __uint_as_float(v.y << 16), a3 = __uint_as_float(v.y & 0xFFFF0000u);
+            ss[t] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, fmaf(a3, a3, ss[t]))));
           }
         }
       }
-      // packed words of rows g and g+8 from the ring
-      if (!ptx::mbar_wait(full(slot), (s / S) & 1, err)) break;
-      uint32_t wa[B + 1], wb[B + 1];
-      const uint8_t* st = tsmem + slot * kStageBytes + warp * kChunkBytes + tig * 4 * B;
-      lds_words<B>(st + g * 16 * B, wa);
-      lds_words<B>(st + (g + 8) * 16 * B, wb);
       uint32_t va[P][16], vb[P][16];
-      expand_group<B>(wa, va);
-      expand_group<B>(wb, vb);
-      // Release the stage only once the words are consumed, and order this
-      // thread's generic-proxy reads before the TMA (async-proxy) writes that
-      // will refill the slot.  Without the fence a refill was observed to land
-      // before the reads of the previous stage in this slot had completed.
-      ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(empty(slot));
+      if constexpr (PAIRED) {
+        expand_paired<B>(wa, va);
+        expand_paired<B>(wb, vb);
+      } else {
+        expand_group<B>(wa, va);
+        expand_group<B>(wb, vb);
+      }
+      if (release) {
+        // Release the stage once its words are in registers, ordering this
+        // thread's generic-proxy reads before the TMA (async-proxy) writes
+        // that will refill the slot.
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(rel_bar);
+      }
       if (active) {
+        if constexpr (!PAIRED) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) permute_x<B>(xw[nt]);
+          for (int nt = 0; nt < NT; ++nt) permute_x<B>(xw[nt]);
+        }
 #pragma unroll
         for (int s2 = 0; s2 < 8; ++s2)
 #pragma unroll
           for (int part = 0; part < P; ++part)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
-              mma_bf16(acc[nt], va[part][2 * s2], vb[part][2 * s2], va[part][2 * s2 + 1],
+              mma_bf16(acc[(s2 * P + part) & 1][nt], va[part][2 * s2], vb[part][2 * s2], va[part][2 * s2 + 1],
                        vb[part][2 * s2 + 1], xw[nt][2 * s2], xw[nt][2 * s2 + 1]);
+      }
+    };
+
+    int slot = 0;
+    uint32_t phase = 0;
+    uint32_t st_off = 0;
+    for (int s = 0; s < n_stages; ++s) {
+      if (!ptx::mbar_wait(full(slot), phase, err)) break;
+      const uint8_t* st = tsmem + st_off;
+      const int c_first = cb + kSC * s + warp * kCH;
+#pragma unroll
+      for (int h = 0; h < kCH; ++h)
+        chunk(st, warp * kCH + h, c_first + h < ce, h == kCH - 1, empty(slot));
+      st_off += st_bytes;
+      if (++slot == S) {
+        slot = 0;
+        phase ^= 1u;
+        st_off = 0;
       }
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) red[warp][nt][lane][q] = acc[nt][q];
+      for (int q = 0; q < 4; ++q) red[warp][nt][lane][q] = acc[0][nt][q] + acc[1][nt][q];
     if (NORM) {
 #pragma unroll
       for (int t = 0; t < NS; ++t) {
@@ -319,6 +370,8 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t* __re
       const int ra = r0 + g, rb = r0 + g + 8;
       const float sca = ra < N ? __ldg(scales + ra) : 0.0f;
       const float scb = rb < N ? __ldg(scales + rb) : 0.0f;
+      // y may be read by the previous kernel in the stream
+      asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -369,23 +422,36 @@ int cluster_size(int tiles, int chunks, int num_sms) {
   return best;
 }
 
-template <int B, int NT, bool NORM>
+template <int B, int NT, bool NORM, bool PAIRED>
 cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
                     uint16_t* y, bool pdl, int32_t* err, cudaStream_t stream) {
   auto encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
   const int64_t rb = 16 * ((static_cast<int64_t>(K) * B + 127) / 128);
-  CUtensorMap tmap;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(N)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(rb)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(16 * B), 16};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides,
-                       box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto kern = gemv_tma_kernel<B, NT, NORM>;
-  const size_t smem = static_cast<size_t>(ring_stages<B>()) * 4 * 16 * 16 * B;
+  CUtensorMap tmap_w, tmap_x;
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(N)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(rb)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(16 * B), 16};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(M)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  auto kern = gemv_tma_kernel<B, NT, NORM, PAIRED>;
+  const int S = ring_stages(B, M);
+  const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M);
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   const int tiles = (N + 15) / 16;
@@ -410,45 +476,55 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
   }
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, tmap, x, M, scales, N, K, y, err);
+  return cudaLaunchKernelEx(&cfg, kern, tmap_w, tmap_x, M, scales, N, K, y, S, err);
 }
 
-template <int B>
+template <int B, bool PAIRED>
 cudaError_t tma_bits(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
                      uint16_t* y, bool norm, bool pdl, int32_t* err, cudaStream_t stream) {
-  if (norm) return run_tma<B, 1, true>(x, M, packed, scales, N, K, y, pdl, err, stream);  // M <= 8
-  if (M <= 8) return run_tma<B, 1, false>(x, M, packed, scales, N, K, y, pdl, err, stream);
-  if (M <= 16) return run_tma<B, 2, false>(x, M, packed, scales, N, K, y, pdl, err, stream);
-  return run_tma<B, 4, false>(x, M, packed, scales, N, K, y, pdl, err, stream);
+  if (norm) return run_tma<B, 1, true, PAIRED>(x, M, packed, scales, N, K, y, pdl, err, stream);  // M <= 8
+  if (M <= 8) return run_tma<B, 1, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, err, stream);
+  if (M <= 16) return run_tma<B, 2, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, err, stream);
+  return run_tma<B, 4, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, err, stream);
+}
+
+template <bool PAIRED>
+cudaError_t tma_layout(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int bits, int N,
+                       int K, uint16_t* y, bool norm, bool pdl, int32_t* err, cudaStream_t stream) {
+  switch (bits) {
+    case 4: return tma_bits<4, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 5: return tma_bits<5, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 6: return tma_bits<6, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 7: return tma_bits<7, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 8: return tma_bits<8, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 9: return tma_bits<9, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 10: return tma_bits<10, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 11: return tma_bits<11, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 12: return tma_bits<12, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 13: return tma_bits<13, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 14: return tma_bits<14, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 15: return tma_bits<15, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
 
-bool gemv_tma_supported(int64_t M, int64_t N, int64_t K, bool norm) {
+bool gemv_tma_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, bool norm) {
+  // TMA of x needs a 16-byte aligned base and a row pitch that is a multiple
+  // of 16 bytes
   return M >= 1 && M <= 32 && (!norm || M <= kNormMaxM) && N >= 1 && K >= 1 && N < (1 << 30) &&
-         tensor_map_encoder() != nullptr;
+         K % 8 == 0 && (reinterpret_cast<uintptr_t>(x) & 15) == 0 && tensor_map_encoder() != nullptr;
 }
 
-cudaError_t launch_gemv_tma(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+cudaError_t launch_gemv_tma(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
                             int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, bool pdl,
                             cudaStream_t stream) {
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   int32_t* err = device_error_word();
-  switch (bits) {
-    case 4: return tma_bits<4>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 5: return tma_bits<5>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 6: return tma_bits<6>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 7: return tma_bits<7>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 8: return tma_bits<8>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 9: return tma_bits<9>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 10: return tma_bits<10>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 11: return tma_bits<11>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 12: return tma_bits<12>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 13: return tma_bits<13>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 14: return tma_bits<14>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    case 15: return tma_bits<15>(x, m, packed, scales, n, k, y, norm, pdl, err, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  if (layout == kLayoutPaired)
+    return tma_layout<true>(x, m, packed, scales, bits, n, k, y, norm, pdl, err, stream);
+  return tma_layout<false>(x, m, packed, scales, bits, n, k, y, norm, pdl, err, stream);
 }
 
 }  // namespace mpw

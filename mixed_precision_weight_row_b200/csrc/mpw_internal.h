@@ -13,6 +13,11 @@ namespace mpw {
 constexpr int kMinBits = 4;
 constexpr int kMaxBits = 15;
 
+// Packed layouts (the values of mpw_layout): canonical LSB-first stream, and
+// the paired-halves re-ordering of the same bits (K % 32 == 0).
+constexpr int kLayoutCanonical = 0;
+constexpr int kLayoutPaired = 1;
+
 // Words (uint32) of one canonical packed row: 4 * ceil(K*b/128).
 inline int64_t row_words(int64_t K, int bits) { return 4 * ((K * bits + 127) / 128); }
 
@@ -42,11 +47,15 @@ cudaError_t launch_unpack(const uint8_t* packed, int64_t N, int64_t K, int bits,
                           int16_t* codes, cudaStream_t stream);
 cudaError_t launch_dequantize(const uint8_t* packed, const float* scales, int64_t N,
                               int64_t K, int bits, float* W_hat, cudaStream_t stream);
+// Canonical <-> paired-halves re-ordering (K % 32 == 0; in == out allowed).
+cudaError_t launch_repack(const uint8_t* in, int64_t N, int64_t K, int bits, uint8_t* out,
+                          bool to_paired, cudaStream_t stream);
 
-// gemv.cu: decode linear y[M, N] for any M (tensor-core kernel in passes of
-// 32 tokens; CUDA-core kernels for shapes it does not take).
+// gemv.cu: decode linear y[M, N] for any M (tensor-core kernels in passes of
+// 32 tokens; CUDA-core kernels for canonical shapes they do not take).  The
+// paired layout needs a shape the TMA kernel takes (checked by the caller).
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* scales,
-                        int bits, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                        int bits, int layout, int64_t M, int64_t N, int64_t K, uint16_t* y,
                         bool norm_input, cudaStream_t stream);
 // The CUDA-core decode kernels alone (x in registers for K <= 17408, else x
 // staged in shared memory), in passes of two tokens.
@@ -61,17 +70,18 @@ cudaError_t launch_gemv_mma(const uint16_t* x, const uint8_t* packed, const floa
                             int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, bool pdl,
                             cudaStream_t stream);
 
-// gemv_tma.cu: decode linear with the packed stream staged by TMA in a
-// shared-memory ring (the default decode kernel for M <= 32).
-bool gemv_tma_supported(int64_t M, int64_t N, int64_t K, bool norm);
+// gemv_tma.cu: decode linear with the packed stream and x staged by TMA in a
+// shared-memory ring (the default decode kernel for M <= 32; needs K % 8 == 0
+// and a 16-byte aligned x).
+bool gemv_tma_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, bool norm);
 cudaError_t launch_gemv_tma(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
-                            int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, bool pdl,
-                            cudaStream_t stream);
+                            int layout, int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm,
+                            bool pdl, cudaStream_t stream);
 
 // gemm.cu: tcgen05 prefill GEMM; returns cudaErrorNotSupported for shapes it
 // does not take (the caller then uses the GEMV path).
 cudaError_t launch_gemm(const uint16_t* x, const uint8_t* packed, const float* scales,
-                        int bits, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                        int bits, int layout, int64_t M, int64_t N, int64_t K, uint16_t* y,
                         int32_t* dev_error, cudaStream_t stream);
 bool gemm_supported(int64_t M, int64_t N, int64_t K);
 

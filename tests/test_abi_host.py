@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("mpw_quantize_pack", "mpw_unpack", "mpw_dequantize", "mpw_qlinear",
                  "mpw_qlinear_path", "mpw_recipe_run", "mpw_packed_row_bytes",
-                 "mpw_status_str", "mpw_version", "mpw_device_error"):
+                 "mpw_status_str", "mpw_version", "mpw_device_error", "mpw_repack",
+                 "mpw_qlinear_ex"):
         assert want in names
 
 
@@ -101,6 +102,32 @@ def test_qlinear_validation():
     assert L.mpw_qlinear_path(A16, A16B, A16, 5, 1, 4, 4, A16, -1, 0) == mpw.MPW_E_INVALID_ARG
 
 
+def test_repack_validation():
+    L = mpw.lib
+    assert L.mpw_repack(A16, 4, 64, 3, 0, 1, A16B, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    assert L.mpw_repack(0, 4, 64, 5, 0, 1, A16B, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_repack(A16, 4, 64, 5, 0, 1, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_repack(A16, 4, 48, 5, 0, 1, A16B, 0) == mpw.MPW_E_INVALID_ARG      # K % 32 != 0
+    assert L.mpw_repack(A16, 0, 64, 5, 0, 1, A16B, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_repack(A16, 4, 64, 5, 1, 1, A16B, 0) == mpw.MPW_E_INVALID_ARG      # same layout
+    assert L.mpw_repack(A16, 4, 64, 5, 0, 2, A16B, 0) == mpw.MPW_E_INVALID_ARG      # unknown layout
+    assert L.mpw_repack(A16, 4, 64, 5, -1, 1, A16B, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_repack(A16 + 8, 4, 64, 5, 0, 1, A16B, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_repack(A16, 4, 64, 5, 0, 1, A16B + 4, 0) == mpw.MPW_E_MISALIGNED
+    # partial overlap (in place is allowed, a shifted copy is not)
+    assert L.mpw_repack(A16, 4, 64, 5, 0, 1, A16 + 16, 0) == mpw.MPW_E_INVALID_ARG
+
+
+def test_qlinear_ex_validation():
+    L = mpw.lib
+    assert L.mpw_qlinear_ex(A16, A16B, A16, 5, 2, 1, 4, 64, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_ex(A16, A16B, A16, 5, -1, 1, 4, 64, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_ex(A16, A16B, A16, 5, 1, 1, 4, 48, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_ex(A16 + 2, A16B, A16, 5, 1, 1, 4, 64, A16, 0, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_qlinear_ex(A16, A16B, A16, 5, 1, 1, 4, 64, A16, 3, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_ex(A16, A16B, A16, 2, 1, 1, 4, 64, A16, 0, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+
+
 def _layers(*specs):
     arr = (mpw._Linear * len(specs))()
     for i, s in enumerate(specs):
@@ -125,6 +152,12 @@ def test_recipe_run_validation():
     assert L.mpw_recipe_run(_layers(good, (A16, A16B, 8, 0, 6, 1, 2, 0)), 2, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
     nulls = (ctypes.c_void_p * 3)(A16, 0, A16B)
     assert L.mpw_recipe_run(_layers(good), 1, nulls, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    # layouts: unknown value, reserved field, K % 32 for paired, x alignment for paired
+    assert L.mpw_recipe_run(_layers((A16, A16B, 8, 64, 6, 0, 1, 0, 2, 0)), 1, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_run(_layers((A16, A16B, 8, 64, 6, 0, 1, 0, 0, 1)), 1, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_run(_layers((A16, A16B, 8, 48, 6, 0, 1, 0, 1, 0)), 1, slots, 3, 1, 0) == mpw.MPW_E_INVALID_ARG
+    odd_slots = (ctypes.c_void_p * 3)(A16 + 2, A16B, A16 + 0x100)
+    assert L.mpw_recipe_run(_layers((A16, A16B, 8, 64, 6, 0, 1, 0, 1, 0)), 1, odd_slots, 3, 1, 0) == mpw.MPW_E_MISALIGNED
 
 
 def test_device_error_rejects_null():

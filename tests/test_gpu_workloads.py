@@ -7,6 +7,10 @@
   quantizer and the linear run at full size in the configuration the benchmark
   uses; a seeded sample of rows is compared (each output column depends on one
   row of W only, so the oracle can compute the sampled columns one by one).
+* prefill (x 2048x5120; 17408x5120 and 5120x5120, b in {5,6,8,10,12}): the
+  tensor-core GEMM on sampled rows.
+Each linear runs on the canonical rows and on their paired-halves re-ordering
+(made on the GPU and compared with the oracle's byte for byte).
 """
 import numpy as np
 import pytest
@@ -62,12 +66,15 @@ def test_decode_workload(mpw, decode_w, b):
     p_ref = oracle.pack(q, b)
     assert np.array_equal(scales.cpu().numpy().view(np.uint32), s.view(np.uint32))
     assert np.array_equal(packed.cpu().numpy(), p_ref)
+    paired = mpw.repack(packed, c["K"], b)
+    assert np.array_equal(paired.cpu().numpy(), oracle.pack_paired(q, b))
     for M in c["Ms"]:
         x = wl.gen_x(M, c["K"], c["x_seed"])
-        y = mpw.qlinear(x.cuda(), packed, scales, b)
         y_ref, bound = oracle.qlinear_ref(x.float().numpy(), q, s)
-        ok = oracle.check_qlinear(y.float().cpu().numpy(), y_ref, bound)
-        assert ok.all(), f"M={M}: {(~ok).sum()} outputs out of bound"
+        for layout, p in (("canonical", packed), ("paired", paired)):
+            y = mpw.qlinear(x.cuda(), p, scales, b, layout=layout)
+            ok = oracle.check_qlinear(y.float().cpu().numpy(), y_ref, bound)
+            assert ok.all(), f"{layout} M={M}: {(~ok).sum()} outputs out of bound"
 
 
 @pytest.mark.parametrize("name,N,K", wl.MLP27B["shapes"][1:], ids=["gate", "down"])
@@ -83,12 +90,15 @@ def test_mlp27b_workload_sampled(mpw, name, N, K, b):
     p_gpu = packed.cpu().numpy()[rows]
     assert np.array_equal(p_gpu, oracle.pack(q, b))
     assert np.array_equal(scales.cpu().numpy()[rows].view(np.uint32), s.view(np.uint32))
+    paired = mpw.repack(packed, K, b)
+    assert np.array_equal(paired.cpu().numpy()[rows], oracle.pack_paired(q, b))
     for M in c["Ms"]:
         x = wl.gen_x(M, K, c["x_seed"])
-        y = mpw.qlinear(x.cuda(), packed, scales, b).float().cpu().numpy()[:, rows]
         y_ref, bound = oracle.qlinear_ref(x.float().numpy(), q, s)
-        ok = oracle.check_qlinear(y, y_ref, bound)
-        assert ok.all(), f"M={M}: {(~ok).sum()} sampled outputs out of bound"
+        for layout, p in (("canonical", packed), ("paired", paired)):
+            y = mpw.qlinear(x.cuda(), p, scales, b, layout=layout).float().cpu().numpy()[:, rows]
+            ok = oracle.check_qlinear(y, y_ref, bound)
+            assert ok.all(), f"{layout} M={M}: {(~ok).sum()} sampled outputs out of bound"
 
 
 @pytest.mark.parametrize("name,N,K", wl.PREFILL["shapes"], ids=["up", "o"])
@@ -99,12 +109,14 @@ def test_prefill_workload_sampled(mpw, name, N, K, b):
     W = wl.gen_weight(N, K, c["sigma"], c["w_seed"])
     x = wl.gen_x(c["M"], K, c["x_seed"])
     packed, scales = mpw.quantize_pack(torch.from_numpy(W).cuda(), b)
-    y = mpw.qlinear(x.cuda(), packed, scales, b)          # M = 2048 -> tensor-core GEMM
-    torch.cuda.synchronize()
     rng = np.random.default_rng(321)
     rows = np.unique(np.concatenate([[0, 127, 128, N - 1], rng.choice(N, 124, replace=False)]))
     q, s = oracle.quantize(W[rows], b)
     y_ref, bound = oracle.qlinear_ref(x.float().numpy(), q, s)
-    ok = oracle.check_qlinear(y.float().cpu().numpy()[:, rows], y_ref, bound)
-    assert ok.all(), f"{(~ok).sum()} sampled outputs out of bound"
+    for layout in ("canonical", "paired"):
+        p = packed if layout == "canonical" else mpw.repack(packed, K, b)
+        y = mpw.qlinear(x.cuda(), p, scales, b, layout=layout)          # M = 2048 -> tensor-core GEMM
+        torch.cuda.synchronize()
+        ok = oracle.check_qlinear(y.float().cpu().numpy()[:, rows], y_ref, bound)
+        assert ok.all(), f"{layout}: {(~ok).sum()} sampled outputs out of bound"
     assert mpw.device_error() == 0
