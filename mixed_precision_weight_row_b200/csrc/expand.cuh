@@ -239,6 +239,67 @@ __device__ __forceinline__ void expand_paired(const uint32_t (&w)[B + 1], uint32
   paired_all<B>(w, v, std::make_integer_sequence<int, 16>{});
 }
 
+// ---------------------------------------------------------------------------
+// Adjacent-pair expansion for the prefill GEMM, whose A operand in tensor
+// memory holds codes (2i, 2i+1) of a group in one 32-bit column.  A code is
+// fed whole when it is exact in bf16 (b <= 9) and as lo7 + 128*hi otherwise
+// (two MMAs into one accumulator); b = 8, 9 and the high part of b = 15 are
+// assembled from two magic fields with a second bf16x2 FMA.
+// ---------------------------------------------------------------------------
+
+template <int B>
+struct GemmParts {
+  static constexpr int parts = B <= 9 ? 1 : 2;
+};
+
+// Field [F0, F0+NB) of codes 2I and 2I+1 as bf16 values 128 + field, for
+// either layout.
+template <int B, bool PAIRED, int I, int F0, int NB, bool SIGNED>
+__device__ __forceinline__ uint32_t field2(const uint32_t (&w)[B + 1]) {
+  if constexpr (PAIRED) {
+    return paired_field<B, I, F0, NB, SIGNED>(w);
+  } else {
+    return adj_pair<B, F0, NB, (SIGNED ? (1u << (NB - 1)) : 0u)>(window<B>(w, 2 * I * B));
+  }
+}
+
+template <int B, bool PAIRED, int I>
+__device__ __forceinline__ void gemm_pair(const uint32_t (&w)[B + 1], uint32_t (&v)[GemmParts<B>::parts][16]) {
+  const uint32_t one = pair_of(1);
+  if constexpr (B <= 7) {
+    v[0][I] = bf2_fma(field2<B, PAIRED, I, 0, B, true>(w), one, pair_of(-(128 + (1 << (B - 1)))));
+  } else if constexpr (B <= 9) {
+    // q = lo7 + 128 * hi fits bf16: t = 128 * hi - 128, then (128 + lo7) + t
+    const uint32_t t = bf2_fma(field2<B, PAIRED, I, 7, B - 7, true>(w), pair_of(128),
+                               pair_of(-128 * (129 + (1 << (B - 8)))));
+    v[0][I] = bf2_fma(field2<B, PAIRED, I, 0, 7, false>(w), one, t);
+  } else if constexpr (B <= 14) {
+    v[0][I] = bf2_fma(field2<B, PAIRED, I, 0, 7, false>(w), one, pair_of(-128));
+    v[1][I] = bf2_fma(field2<B, PAIRED, I, 7, B - 7, true>(w), pair_of(128),
+                      pair_of(-128 * (128 + (1 << (B - 8)))));
+  } else {
+    // 128 * hi with hi = mid7 + 128 * (top' - 1): t = 16384 * top' - 32768,
+    // then 128 * (128 + mid7) + t
+    v[0][I] = bf2_fma(field2<B, PAIRED, I, 0, 7, false>(w), one, pair_of(-128));
+    const uint32_t t = bf2_fma(field2<B, PAIRED, I, 14, 1, true>(w), pair_of(16384),
+                               pair_of(-16384 * 128 - 32768));
+    v[1][I] = bf2_fma(field2<B, PAIRED, I, 7, 7, false>(w), pair_of(128), t);
+  }
+}
+
+template <int B, bool PAIRED, int... I>
+__device__ __forceinline__ void gemm_all(const uint32_t (&w)[B + 1], uint32_t (&v)[GemmParts<B>::parts][16],
+                                         std::integer_sequence<int, I...>) {
+  (gemm_pair<B, PAIRED, I>(w, v), ...);
+}
+
+// One 32-code group -> 16 adjacent bf16x2 pairs per part (exact values).
+template <int B, bool PAIRED>
+__device__ __forceinline__ void gemm_expand_group(const uint32_t (&w)[B + 1],
+                                                  uint32_t (&v)[GemmParts<B>::parts][16]) {
+  gemm_all<B, PAIRED>(w, v, std::make_integer_sequence<int, 16>{});
+}
+
 __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
   asm volatile(

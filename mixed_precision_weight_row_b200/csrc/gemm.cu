@@ -8,134 +8,123 @@
 //
 // One CTA computes a 128-row (W) x 256-token (x) tile of y^T with
 // tcgen05.mma.cta_group::1.kind::f16, M=128, N=256, K=16:
+//   * Packed weights move in blocks of 128 codes (16*B bytes per row): warp 3
+//     copies them with 16-byte cp.async (consecutive lanes take consecutive
+//     16-byte units of a row, so each warp instruction reads whole lines)
+//     into a shared-memory ring whose row pitch is padded to an odd number
+//     of 16-byte units, so the converters' 16-byte reads are free of bank
+//     conflicts; completion reaches an mbarrier through
+//     cp.async.mbarrier.arrive.
 //   * A = 128 weight rows x 16 codes, held in TENSOR MEMORY.  Converter warps
-//     (8 warps, one weight row per thread per half k-block) read the packed
-//     row straight from global memory, expand each b-bit code to an exact
-//     bf16 value and store it with tcgen05.st, so the expanded weights never
-//     touch shared memory.  Codes up to 9 bits are exact in bf16; wider codes
-//     are split q = 256*hi + lo (lo = q & 255, both parts exact in bf16) and
-//     issued as two MMAs into the same accumulator.
-//   * B = 256 tokens x 16 of x, loaded by TMA (128-byte swizzle, K-major) into
-//     a 6-stage shared-memory ring.
+//     (two groups of four, alternating weight blocks; one row per thread)
+//     expand each pair of codes to an exact bf16x2 value with a bit-field
+//     magic number and one bf16x2 FMA (expand.cuh) and store it with
+//     tcgen05.st.  Codes up to 9 bits are fed whole; wider codes as
+//     lo7 + 128*hi, two MMAs into the same accumulator, so no code is ever
+//     rounded.
+//   * B = 256 tokens x 64 of x, loaded by TMA (128-byte swizzle, K-major)
+//     into a 4- or 5-stage ring.
 //   * D = fp32 accumulator, 128 lanes x 256 columns of tensor memory.
-// Warp roles: 0 = TMA producer, 1 = MMA issuer, 2 = tensor-memory allocator,
-// 4..11 = converters, then the epilogue (tcgen05.ld, row scale, bf16 store).
-// Every mbarrier wait is bounded; on time-out the kernel records an error in
-// the device error word and every role falls through to the final barrier.
+// Warp roles: 0 = x TMA producer, 1 = MMA issuer, 2 = tensor-memory
+// allocator, 3 = weight producer, 4..11 = converters, then the epilogue
+// (tcgen05.ld, row scale, bf16 store).  Every mbarrier wait is bounded; on
+// time-out the kernel records an error in the device error word and every
+// role falls through to the final barrier.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "expand.cuh"
 #include "mpw_internal.h"
 #include "tc_ptx.cuh"
 
 namespace mpw {
 namespace {
 
+using namespace dec;
+
 constexpr int BM = 128;          // weight rows per CTA (MMA M)
 constexpr int BN = 256;          // tokens per CTA (MMA N)
-constexpr int BK = 64;           // codes per k-block (one 128-byte swizzle atom of bf16)
-constexpr int SX = 6;            // x stages in shared memory
-constexpr int SA = 4;            // A stages in tensor memory
+constexpr int BK = 64;           // codes per x stage (one 128-byte swizzle atom of bf16)
+constexpr int WB = 128;          // codes per weight block
+constexpr int SW = 3;            // weight stages in shared memory
 constexpr int kThreads = 384;    // 12 warps
 constexpr int kConvWarp0 = 4;    // first converter warp
 constexpr uint32_t kXStageBytes = BN * BK * 2;   // 32 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = BN;                // fp32 accumulator columns
-constexpr size_t kSmemBytes = SX * kXStageBytes + 1024 /*align slack*/ + 256 /*barriers*/;
 
 template <int B>
 struct GemmCode {
-  static constexpr bool HL = B > 9;                    // hi/lo split needed
-  static constexpr uint32_t ACOLS = HL ? 64 : 32;      // tensor-memory columns per A stage
+  // x stages in shared memory: as many as fit beside the weight stages
+  static constexpr int SX = B <= 8 ? 5 : 4;
+  static constexpr int P = GemmParts<B>::parts;              // MMAs per k-step
+  static constexpr uint32_t ACOLS = 64u * P;                 // tensor-memory columns per A stage
+  static constexpr int SA = static_cast<int>((kTmemCols - kAccCols) / ACOLS);
+  // row pitch of a weight stage: 16*B bytes padded to an odd number of
+  // 16-byte units
+  static constexpr uint32_t PITCH = 16u * (B % 2 == 1 ? B : B + 1);
+  static constexpr uint32_t WSTAGE = BM * PITCH;
+  static constexpr size_t SMEM = SX * kXStageBytes + SW * WSTAGE + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(SMEM <= 232448, "shared memory per block");
 };
 
-// Code j (0..31) of a 32-code group as an exact fp32 integer.
-template <int B>
-__device__ __forceinline__ float code_f32(const uint32_t (&w)[B + 1], int j) {
-  const int o = j * B;
-  const int i = o >> 5, r = o & 31;
-  uint32_t t;
-  if (r == 0) t = w[i];
-  else if (r + B <= 32) t = w[i] >> r;
-  else t = __funnelshift_r(w[i], w[i + 1], r);
-  constexpr uint32_t kMask = (1u << B) - 1u;
-  constexpr uint32_t kMagic = 0x4B000000u | (1u << (B - 1));
-  constexpr float kOffset = 8388608.0f + static_cast<float>(1 << (B - 1));
-  return __uint_as_float((t & kMask) ^ kMagic) - kOffset;
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
 }
 
-// Code j (0..31) of a 32-code group of a paired-halves row: even codes form
-// the stream in the low half-words, odd codes the stream in the high ones.
-template <int B>
-__device__ __forceinline__ float code_f32_paired(const uint32_t (&w)[B + 1], int j) {
-  const int o = (j >> 1) * B;
-  const int h = o >> 4, r = o & 15;
-  // half-words h and h+1 of the code's stream as one 32-bit window
-  const uint32_t win = __byte_perm(w[h], w[h + 1], (j & 1) ? 0x7632 : 0x5410);
-  constexpr uint32_t kMask = (1u << B) - 1u;
-  constexpr uint32_t kMagic = 0x4B000000u | (1u << (B - 1));
-  constexpr float kOffset = 8388608.0f + static_cast<float>(1 << (B - 1));
-  return __uint_as_float(((win >> r) & kMask) ^ kMagic) - kOffset;
-}
-
-template <int B, bool PAIRED>
-__device__ __forceinline__ float code_at(const uint32_t (&w)[B + 1], int j) {
-  if constexpr (PAIRED) return code_f32_paired<B>(w, j);
-  else return code_f32<B>(w, j);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-template <int B>
-__device__ __forceinline__ void load_group(const uint32_t* __restrict__ rowp, int g, int rw,
-                                           bool row_ok, uint32_t (&w)[B + 1]) {
-  const bool full = row_ok && (g + 1) * B <= rw;
-#pragma unroll
-  for (int i = 0; i < B; ++i) {
-    const int idx = g * B + i;
-    w[i] = full ? __ldg(rowp + idx) : ((row_ok && idx < rw) ? __ldg(rowp + idx) : 0u);
-  }
-  w[B] = 0u;
+// Arrives on the mbarrier once every cp.async this thread issued has landed
+// (the arrival is counted in the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 template <int B, bool PAIRED>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ packed,
-            const float* __restrict__ scales, uint16_t* __restrict__ y, int M, int N, int K, int rw,
+            const float* __restrict__ scales, uint16_t* __restrict__ y, int M, int N, int K, int rb,
             int32_t* err) {
   using C = GemmCode<B>;
+  constexpr int P = C::P;
+  constexpr int SA = C::SA;
+  constexpr int SX = C::SX;
   extern __shared__ uint8_t gsmem_raw[];
   const uint32_t raw = ptx::smem_addr(gsmem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;       // 1024-aligned for the 128-byte swizzle
   uint8_t* gsmem = gsmem_raw + (base - raw);
   const uint32_t xs0 = base;                           // SX x stages
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gsmem + SX * kXStageBytes);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * SX + 2 * SA + 1);
+  const uint32_t ws0 = base + SX * kXStageBytes;       // SW weight stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gsmem + SX * kXStageBytes + SW * C::WSTAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * SX + 2 * SW + 2 * SA + 1);
   const uint32_t bar0 = ptx::smem_addr(bars);
   auto full_x = [&](int s) { return bar0 + 8u * s; };
   auto empty_x = [&](int s) { return bar0 + 8u * (SX + s); };
-  auto full_a = [&](int s) { return bar0 + 8u * (2 * SX + s); };
-  auto empty_a = [&](int s) { return bar0 + 8u * (2 * SX + SA + s); };
-  const uint32_t acc_full = bar0 + 8u * (2 * SX + 2 * SA);
+  auto full_w = [&](int s) { return bar0 + 8u * (2 * SX + s); };
+  auto empty_w = [&](int s) { return bar0 + 8u * (2 * SX + SW + s); };
+  auto full_a = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SW + s); };
+  auto empty_a = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SW + SA + s); };
+  const uint32_t acc_full = bar0 + 8u * (2 * SX + 2 * SW + 2 * SA);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BM;
   const int m0 = blockIdx.y * BN;
-  const int KB = (K + BK - 1) / BK;
+  const int KB = (K + BK - 1) / BK;      // x stages
+  const int WBs = (K + WB - 1) / WB;     // weight blocks
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SX; ++s) {
       ptx::mbar_init(full_x(s), 1);
       ptx::mbar_init(empty_x(s), 1);
     }
+    for (int s = 0; s < SW; ++s) {
+      ptx::mbar_init(full_w(s), 32);        // the weight producer's lanes
+      ptx::mbar_init(empty_w(s), 128);      // one converter group
+    }
     for (int s = 0; s < SA; ++s) {
-      ptx::mbar_init(full_a(s), 32 * (kThreads / 32 - kConvWarp0));
+      ptx::mbar_init(full_a(s), 128);       // one converter group
       ptx::mbar_init(empty_a(s), 1);
     }
     ptx::mbar_init(acc_full, 1);
@@ -154,84 +143,114 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restric
   const uint32_t tmem_a = tmem + kAccCols;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- x TMA producer ----------------
     if (lane == 0) {
+      int issued = 0;
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % SX;
-        const uint32_t ph = (kb / SX) & 1;
-        if (!ptx::mbar_wait(empty_x(s), ph ^ 1, err)) break;
+        if (!ptx::mbar_wait(empty_x(s), ((kb / SX) & 1) ^ 1, err)) break;
         ptx::mbar_arrive_expect_tx(full_x(s), kXStageBytes);
         ptx::tma_load_2d(xs0 + s * kXStageBytes, &tmap_x, full_x(s), kb * BK, m0);
+        issued = kb + 1;
       }
+      // nothing may still be landing in shared memory when the CTA exits
+      for (int kb = max(0, issued - SX); kb < issued; ++kb) ptx::mbar_wait(full_x(kb % SX), (kb / SX) & 1, err);
     }
+  } else if (warp == 3) {
+    // ---------------- weight producer: 16-byte cp.async ----------------
+    int issued = 0;
+    for (int wb = 0; wb < WBs; ++wb) {
+      const int s = wb % SW;
+      bool ok = true;
+      if (lane == 0) ok = ptx::mbar_wait(empty_w(s), ((wb / SW) & 1) ^ 1, err);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      // the last block of a row may be shorter (the row ends at rb bytes)
+      const int units = min(B, (rb - wb * 16 * B) / 16);
+      const uint8_t* blk = packed + static_cast<size_t>(wb) * 16 * B;
+      const uint32_t dst0 = ws0 + s * C::WSTAGE;
+#pragma unroll 4
+      for (int idx = lane; idx < BM * B; idx += 32) {
+        const int r = idx / B, u = idx - r * B;
+        if (u < units) {
+          const int n = min(n0 + r, N - 1);   // rows past N: any valid row (their outputs are not stored)
+          cp_async16(dst0 + r * C::PITCH + u * 16, blk + static_cast<size_t>(n) * rb + u * 16);
+        }
+      }
+      cp_async_arrive(full_w(s));
+      issued = wb + 1;
+    }
+    // nothing may still be landing in shared memory when the CTA exits
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (lane == 0)
+      for (int wb = max(0, issued - SW); wb < issued; ++wb) ptx::mbar_wait(full_w(wb % SW), (wb / SW) & 1, err);
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, BN);
       bool ok = true;
       for (int kb = 0; kb < KB && ok; ++kb) {
-        const int sx = kb % SX, sa = kb % SA;
-        ok = ptx::mbar_wait(full_x(sx), (kb / SX) & 1, err) &&
-             ptx::mbar_wait(full_a(sa), (kb / SA) & 1, err);
+        const int sx = kb % SX;
+        const int wb = kb >> 1, h = kb & 1, sa = wb % SA;
+        ok = ptx::mbar_wait(full_x(sx), (kb / SX) & 1, err);
+        if (ok && h == 0) ok = ptx::mbar_wait(full_a(sa), (wb / SA) & 1, err);
         if (!ok) break;
         ptx::tc_fence_after();
         const uint64_t bdesc = ptx::sw128_kmajor_desc(xs0 + sx * kXStageBytes);
-        const uint32_t a_stage = tmem_a + sa * C::ACOLS;
+        const uint32_t a_cols = tmem_a + sa * C::ACOLS + h * 32;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           const uint64_t bd = bdesc + static_cast<uint64_t>(2 * kk);  // +32 bytes along K
-          if (C::HL) {
-            ptx::mma_ts(tmem_acc, a_stage + kk * 8, bd, idesc, (kb | kk) != 0);
-            ptx::mma_ts(tmem_acc, a_stage + 32 + kk * 8, bd, idesc, 1u);
-          } else {
-            ptx::mma_ts(tmem_acc, a_stage + kk * 8, bd, idesc, (kb | kk) != 0);
-          }
+          ptx::mma_ts(tmem_acc, a_cols + kk * 8, bd, idesc, (kb | kk) != 0);
+          if constexpr (P == 2) ptx::mma_ts(tmem_acc, a_cols + 64 + kk * 8, bd, idesc, 1u);
         }
         ptx::mma_commit(empty_x(sx));
-        ptx::mma_commit(empty_a(sa));
+        if (h == 1 || kb == KB - 1) ptx::mma_commit(empty_a(sa));
       }
       ptx::mma_commit(acc_full);
     }
   } else if (warp >= kConvWarp0) {
     // ---------------- converters, then epilogue ----------------
-    const int wg = (warp - kConvWarp0) >> 2;       // which half of each k-block
+    const int wg = (warp - kConvWarp0) >> 2;       // which weight blocks (even / odd)
     const int quad = warp & 3;                     // tensor-memory lane quadrant
     const int r = quad * 32 + lane;                // weight row within the tile
     const int n = n0 + r;
     const bool row_ok = n < N;
-    const uint32_t* rowp = reinterpret_cast<const uint32_t*>(packed) + static_cast<size_t>(row_ok ? n : 0) * rw;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     bool ok = true;
-    uint32_t wcur[B + 1], wnext[B + 1];
-    load_group<B>(rowp, wg, rw, row_ok, wcur);
-    for (int kb = 0; kb < KB; ++kb) {
-      const int s = kb % SA;
-      if (kb + 1 < KB) load_group<B>(rowp, 2 * (kb + 1) + wg, rw, row_ok, wnext);
-      uint32_t va[16], vb[16];
-      if (C::HL) {
+    for (int wb = wg; wb < WBs; wb += 2) {
+      const int ws = wb % SW, sa = wb % SA;
+      ok = ptx::mbar_wait(full_w(ws), (wb / SW) & 1, err);
+      if (!ok) break;
+      // the row's 4 groups: 16*B bytes, read as 16-byte units
+      uint32_t w[4 * B + 1];
+      const uint4* src = reinterpret_cast<const uint4*>(gsmem + SX * kXStageBytes + ws * C::WSTAGE + r * C::PITCH);
 #pragma unroll
-        for (int p = 0; p < 16; ++p) {
-          const float q0 = code_at<B, PAIRED>(wcur, 2 * p), q1 = code_at<B, PAIRED>(wcur, 2 * p + 1);
-          const int i0 = static_cast<int>(q0), i1 = static_cast<int>(q1);
-          const float l0 = static_cast<float>(i0 & 255), l1 = static_cast<float>(i1 & 255);
-          va[p] = pack_bf16x2(q0 - l0, q1 - l1);   // 256 * hi, exact
-          vb[p] = pack_bf16x2(l0, l1);             // lo in [0, 255], exact
-        }
-      } else {
-#pragma unroll
-        for (int p = 0; p < 16; ++p) va[p] = pack_bf16x2(code_at<B, PAIRED>(wcur, 2 * p), code_at<B, PAIRED>(wcur, 2 * p + 1));
+      for (int i = 0; i < B; ++i) {
+        const uint4 v = src[i];
+        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
       }
-      ok = ptx::mbar_wait(empty_a(s), ((kb / SA) & 1) ^ 1, err);
+      w[4 * B] = 0u;
+      // the async-proxy refill of this stage must not overtake these reads
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive(empty_w(ws));
+      ok = ptx::mbar_wait(empty_a(sa), ((wb / SA) & 1) ^ 1, err);
       if (!ok) break;
       ptx::tc_fence_after();
-      const uint32_t col = kAccCols + s * C::ACOLS + wg * 16;
-      ptx::tmem_st16(tmem + lane_addr + col, va);
-      if (C::HL) ptx::tmem_st16(tmem + lane_addr + col + 32, vb);
+      const uint32_t col = tmem + lane_addr + kAccCols + sa * C::ACOLS;
+#pragma unroll
+      for (int g4 = 0; g4 < 4; ++g4) {
+        uint32_t gw[B + 1];
+#pragma unroll
+        for (int i = 0; i <= B; ++i) gw[i] = w[g4 * B + i];
+        uint32_t v[P][16];
+        gemm_expand_group<B, PAIRED>(gw, v);
+        ptx::tmem_st16(col + g4 * 16, v[0]);
+        if constexpr (P == 2) ptx::tmem_st16(col + 64 + g4 * 16, v[1]);
+      }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(full_a(s));
-#pragma unroll
-      for (int i = 0; i <= B; ++i) wcur[i] = wnext[i];
+      ptx::mbar_arrive(full_a(sa));
     }
     if (ok) ok = ptx::mbar_wait(acc_full, 0, err);
     if (ok) {
@@ -267,6 +286,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restric
 template <int B, bool PAIRED>
 cudaError_t run_gemm(const uint16_t* x, const uint8_t* packed, const float* scales, int64_t M,
                      int64_t N, int64_t K, uint16_t* y, int32_t* err, cudaStream_t stream) {
+  using C = GemmCode<B>;
   auto encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap;
@@ -279,20 +299,13 @@ cudaError_t run_gemm(const uint16_t* x, const uint8_t* packed, const float* scal
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
   auto kern = gemm_kernel<B, PAIRED>;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kSmemBytes);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>((N + BM - 1) / BM), static_cast<unsigned>((M + BN - 1) / BN));
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(tmap, packed, scales, y, static_cast<int>(M),
-                                               static_cast<int>(N), static_cast<int>(K),
-                                               static_cast<int>(row_words(K, B)), err);
+  kern<<<grid, kThreads, C::SMEM, stream>>>(tmap, packed, scales, y, static_cast<int>(M), static_cast<int>(N),
+                                            static_cast<int>(K), static_cast<int>(16 * ((K * B + 127) / 128)),
+                                            err);
   return cudaGetLastError();
-}
-
-}  // namespace
-
-bool gemm_supported(int64_t M, int64_t N, int64_t K) {
-  // TMA needs the x row stride (K * 2 bytes) to be a multiple of 16 bytes.
-  return K % 8 == 0 && M >= 1 && N >= 1 && (M + BN - 1) / BN <= 65535;
 }
 
 template <bool PAIRED>
@@ -313,6 +326,13 @@ cudaError_t gemm_layout(const uint16_t* x, const uint8_t* packed, const float* s
     case 15: return run_gemm<15, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+}  // namespace
+
+bool gemm_supported(int64_t M, int64_t N, int64_t K) {
+  // TMA needs the x row stride (K * 2 bytes) to be a multiple of 16 bytes.
+  return K % 8 == 0 && M >= 1 && N >= 1 && (M + BN - 1) / BN <= 65535;
 }
 
 cudaError_t launch_gemm(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,

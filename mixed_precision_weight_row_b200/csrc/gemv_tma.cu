@@ -55,7 +55,6 @@ constexpr int kThreads = (kCW + 1) * 32;
 constexpr int kChunk = 128;             // codes per chunk and row
 constexpr int kNormMaxM = 8;
 constexpr int kMaxStages = 8;
-constexpr uint32_t kRingBudget = 48u * 1024u;
 
 // Bytes of one stage: kSC weight chunks (16 rows x 16*B bytes) followed by
 // kSC x chunks (M tokens x 128 bf16).
@@ -63,14 +62,25 @@ __host__ __device__ constexpr uint32_t stage_bytes(int B, int M) {
   return static_cast<uint32_t>(kSC) * 256u * static_cast<uint32_t>(B + M);
 }
 
-int ring_stages(int B, int M) {
-  // MPW_GEMV_RING_KB overrides the ring budget (tuning aid)
+// Ring depth.  With at most two CTAs per SM, a CTA whose whole K slice fits
+// in kWholeSlice bytes puts every stage of it in flight at once (latency
+// decides); otherwise two stages keep shared memory per CTA small and the
+// number of resident CTAs per SM high (occupancy decides).
+// MPW_GEMV_RING_KB replaces the rule by a fixed budget (tuning aid).
+constexpr uint32_t kWholeSlice = 64u * 1024u;
+
+int ring_stages(int B, int M, int stages_per_cta, bool few_ctas) {
   static const uint32_t budget = [] {
     const char* e = getenv("MPW_GEMV_RING_KB");
     const int v = e ? atoi(e) : 0;
-    return v >= 8 && v <= 192 ? static_cast<uint32_t>(v) * 1024u : kRingBudget;
+    return v >= 8 && v <= 192 ? static_cast<uint32_t>(v) * 1024u : 0u;
   }();
-  const int s = static_cast<int>(budget / stage_bytes(B, M));
+  const uint32_t st = stage_bytes(B, M);
+  int s;
+  if (budget != 0)
+    s = static_cast<int>(budget / st);
+  else
+    s = few_ctas && static_cast<uint32_t>(stages_per_cta) * st <= kWholeSlice ? stages_per_cta : 2;
   return s < 2 ? 2 : (s > kMaxStages ? kMaxStages : s);
 }
 
@@ -450,13 +460,14 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
       return cudaErrorInvalidValue;
   }
   auto kern = gemv_tma_kernel<B, NT, NORM, PAIRED>;
-  const int S = ring_stages(B, M);
-  const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M);
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
-  if (e != cudaSuccess) return e;
   const int tiles = (N + 15) / 16;
   const int chunks = (K + kChunk - 1) / kChunk;
   const int kc = cluster_size(tiles, chunks, device_info().num_sms);
+  const int per_cta = ((chunks + kc - 1) / kc + kSC - 1) / kSC;
+  const int S = ring_stages(B, M, per_cta, tiles * kc <= 2 * device_info().num_sms);
+  const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(tiles * kc));
   cfg.blockDim = dim3(kThreads);
