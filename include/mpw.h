@@ -177,6 +177,30 @@ MPW_API mpw_status mpw_qlinear_ex(const uint16_t* x, const uint8_t* packed, cons
                                   uint16_t* y, int path, mpw_stream_t stream);
 
 /*
+ * Workspace of the decode kernels.  For M <= 32 the fastest decode kernel
+ * splits the (16-row tile, 128-code chunk) units of W evenly over a
+ * persistent grid; a tile shared by two or more CTAs is combined through a
+ * small caller-provided workspace (partial sums and one counter per tile).
+ *   - device memory, 16-byte aligned, at least the size returned below;
+ *   - zero-filled by the caller once before its first use; every call that
+ *     completes leaves it ready for the next one (its counters back at zero);
+ *     after a call that reported MPW_E_TIMEOUT it must be zero-filled again;
+ *   - calls that share one workspace must not run at the same time (calls on
+ *     one stream never do).
+ * mpw_qlinear_workspace_bytes returns the bytes a call with these arguments
+ * needs (0 when it uses no workspace).  A NULL workspace selects the
+ * per-tile decode kernel, which needs none; a non-NULL workspace smaller
+ * than required is an argument error.
+ */
+MPW_API size_t mpw_qlinear_workspace_bytes(int bits, int layout, int64_t M, int64_t N, int64_t K);
+
+/* mpw_qlinear_ex with a decode workspace (see above); same results. */
+MPW_API mpw_status mpw_qlinear_ws(const uint16_t* x, const uint8_t* packed, const float* scales,
+                                  int bits, int layout, int64_t M, int64_t N, int64_t K,
+                                  uint16_t* y, int path, void* workspace, size_t workspace_bytes,
+                                  mpw_stream_t stream);
+
+/*
  * One linear of a recipe stack (DynaQuant "Step 3": every matrix carries its
  * own bit width).  Activations move between caller-owned "slots".
  *   packed, scales, N, K, bits  the quantized matrix (device pointers).
@@ -214,6 +238,16 @@ typedef struct mpw_linear {
 MPW_API mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count,
                           uint16_t* const* slots, int64_t num_slots, int64_t M,
                           mpw_stream_t stream);
+
+/* Workspace bytes for mpw_recipe_run_ws over these layers (the largest any
+ * one of them needs). */
+MPW_API size_t mpw_recipe_workspace_bytes(const mpw_linear* layers, int64_t count, int64_t M);
+
+/* mpw_recipe_run with a decode workspace (see mpw_qlinear_workspace_bytes);
+ * the linears run one after another and share it. */
+MPW_API mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count,
+                                     uint16_t* const* slots, int64_t num_slots, int64_t M,
+                                     void* workspace, size_t workspace_bytes, mpw_stream_t stream);
 
 /*
  * mpw_device_error -- synchronises the current device, returns in *code the

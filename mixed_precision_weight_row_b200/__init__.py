@@ -18,7 +18,7 @@ from dataclasses import dataclass
 __all__ = [
     "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
     "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str",
-    "LAYOUTS",
+    "LAYOUTS", "workspace", "qlinear_workspace_bytes",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmpw.so")
@@ -84,6 +84,15 @@ def _load():
     L.mpw_qlinear_ex.restype = c_int
     L.mpw_repack.argtypes = [vp, i64, i64, c_int, c_int, c_int, vp, vp]
     L.mpw_repack.restype = c_int
+    L.mpw_qlinear_workspace_bytes.argtypes = [c_int, c_int, i64, i64, i64]
+    L.mpw_qlinear_workspace_bytes.restype = ctypes.c_size_t
+    L.mpw_qlinear_ws.argtypes = [vp, vp, vp, c_int, c_int, i64, i64, i64, vp, c_int, vp, ctypes.c_size_t, vp]
+    L.mpw_qlinear_ws.restype = c_int
+    L.mpw_recipe_workspace_bytes.argtypes = [ctypes.POINTER(_Linear), i64, i64]
+    L.mpw_recipe_workspace_bytes.restype = ctypes.c_size_t
+    L.mpw_recipe_run_ws.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp,
+                                    ctypes.c_size_t, vp]
+    L.mpw_recipe_run_ws.restype = c_int
     L.mpw_recipe_run.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp]
     L.mpw_recipe_run.restype = c_int
     L.mpw_device_error.argtypes = [ctypes.POINTER(i32)]
@@ -126,6 +135,32 @@ def _need(t, dtype, name, ndim=None):
         raise ValueError(f"{name} must be contiguous")
     if ndim is not None and t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dims")
+
+
+# Decode workspaces (see mpw_qlinear_workspace_bytes in mpw.h), one per
+# (device, stream): zero-filled when created, grown by replacement.  Calls on
+# one stream are ordered, so they may share it.
+_workspaces = {}
+
+
+def workspace(nbytes: int, stream=None):
+    """A zero-filled decode workspace of at least ``nbytes`` for this stream."""
+    import torch
+
+    if nbytes <= 0:
+        return None
+    dev = torch.cuda.current_device()
+    key = (dev, _stream(stream))
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        size = max(int(nbytes), 1 << 20, 0 if ws is None else 2 * ws.numel())
+        ws = torch.zeros(size, dtype=torch.uint8, device=f"cuda:{dev}")
+        _workspaces[key] = ws
+    return ws
+
+
+def qlinear_workspace_bytes(bits: int, M: int, N: int, K: int, layout: str = "canonical") -> int:
+    return int(lib.mpw_qlinear_workspace_bytes(int(bits), LAYOUTS[layout], int(M), int(N), int(K)))
 
 
 def packed_row_bytes(K: int, bits: int) -> int:
@@ -200,8 +235,12 @@ def repack(packed, K: int, bits: int, layout_in: str = "canonical", layout_out: 
 
 
 def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: str = "canonical",
-            stream=None):
-    """y = x @ (q * s)^T with x bf16 [M, K]; returns y bf16 [M, N]."""
+            stream=None, use_workspace: bool = False):
+    """y = x @ (q * s)^T with x bf16 [M, K]; returns y bf16 [M, N].
+
+    With ``use_workspace`` the decode path (M <= 32) gets this stream's
+    workspace and runs the stream-K kernel; without it (the default, faster
+    on every measured shape) the per-tile kernel."""
     import torch
 
     _need(x, torch.bfloat16, "x", 2)
@@ -216,8 +255,16 @@ def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: st
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(y, torch.bfloat16, "y")
-    _check(lib.mpw_qlinear_ex(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits), LAYOUTS[layout],
-                              M, N, K, y.data_ptr(), PATHS[path], _stream(stream)), "mpw_qlinear")
+    ws, ws_bytes = None, 0
+    if use_workspace:
+        need = qlinear_workspace_bytes(bits, min(M, 32), N, K, layout) if M <= 32 or path == "gemv" else 0
+        if M > 32 and path == "gemv":
+            need = max(need, qlinear_workspace_bytes(bits, M % 32 or 32, N, K, layout))
+        ws = workspace(need, stream)
+        ws_bytes = 0 if ws is None else ws.numel()
+    _check(lib.mpw_qlinear_ws(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits), LAYOUTS[layout],
+                              M, N, K, y.data_ptr(), PATHS[path], None if ws is None else ws.data_ptr(),
+                              ws_bytes, _stream(stream)), "mpw_qlinear")
     return y
 
 
@@ -235,14 +282,19 @@ class Linear:
     layout: str = "canonical"
 
 
-def recipe_run(layers, slots, M: int, stream=None):
+def recipe_run(layers, slots, M: int, stream=None, use_workspace: bool = False):
     """Launch every linear of ``layers`` in order (one kernel each)."""
     arr = (_Linear * len(layers))()
     for i, L in enumerate(layers):
         arr[i] = _Linear(L.packed.data_ptr(), L.scales.data_ptr(), int(L.N), int(L.K), int(L.bits),
                          int(L.in_slot), int(L.out_slot), int(bool(L.norm_input)), LAYOUTS[L.layout], 0)
     ptrs = (ctypes.c_void_p * len(slots))(*[s.data_ptr() for s in slots])
-    _check(lib.mpw_recipe_run(arr, len(layers), ptrs, len(slots), int(M), _stream(stream)),
+    ws, ws_bytes = None, 0
+    if use_workspace:
+        ws = workspace(int(lib.mpw_recipe_workspace_bytes(arr, len(layers), int(M))), stream)
+        ws_bytes = 0 if ws is None else ws.numel()
+    _check(lib.mpw_recipe_run_ws(arr, len(layers), ptrs, len(slots), int(M),
+                                 None if ws is None else ws.data_ptr(), ws_bytes, _stream(stream)),
            "mpw_recipe_run")
 
 

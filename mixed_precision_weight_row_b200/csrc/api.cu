@@ -111,7 +111,7 @@ const char* mpw_status_str(int status) {
   }
 }
 
-int mpw_version(void) { return 200; }
+int mpw_version(void) { return 300; }
 
 size_t mpw_packed_row_bytes(int64_t K, int bits) {
   if (!bits_ok(bits) || K < 1) return 0;
@@ -167,8 +167,11 @@ mpw_status mpw_repack(const uint8_t* in, int64_t N, int64_t K, int bits, int lay
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
-mpw_status mpw_qlinear_ex(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
-                          int64_t M, int64_t N, int64_t K, uint16_t* y, int path, mpw_stream_t stream) {
+namespace {
+
+mpw_status qlinear_impl(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
+                        int64_t M, int64_t N, int64_t K, uint16_t* y, int path, void* ws, size_t ws_bytes,
+                        mpw_stream_t stream) {
   if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
   if (x == nullptr || packed == nullptr || scales == nullptr || y == nullptr || M < 1 || N < 1 ||
       K < 1)
@@ -179,13 +182,34 @@ mpw_status mpw_qlinear_ex(const uint16_t* x, const uint8_t* packed, const float*
   if (paired && K % 32 != 0) return MPW_E_INVALID_ARG;
   if (!aligned(packed, 16) || !aligned(x, paired ? 16 : 2) || !aligned(y, 2) || !aligned(scales, 4))
     return MPW_E_MISALIGNED;
+  if (ws != nullptr && !aligned(ws, 16)) return MPW_E_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool want_gemm = path == MPW_PATH_GEMM || (path == MPW_PATH_AUTO && M > 32);
   if (want_gemm && gemm_supported(M, N, K) && aligned(x, 16)) {
     return from_cuda(launch_gemm(x, packed, scales, bits, layout, M, N, K, y, device_error_word(), s));
   }
   if (path == MPW_PATH_GEMM) return MPW_E_INVALID_ARG;  // shape the GEMM does not take
-  return from_cuda(launch_gemv(x, packed, scales, bits, layout, M, N, K, y, false, s));
+  if (ws != nullptr && ws_bytes < gemv_workspace_bytes(x, bits, layout, M, N, K, false)) return MPW_E_INVALID_ARG;
+  return from_cuda(launch_gemv(x, packed, scales, bits, layout, M, N, K, y, false, ws, ws_bytes, s));
+}
+
+}  // namespace
+
+size_t mpw_qlinear_workspace_bytes(int bits, int layout, int64_t M, int64_t N, int64_t K) {
+  if (!bits_ok(bits) || !layout_ok(layout) || M < 1 || N < 1 || K < 1 || M > 32) return 0;
+  if (N > 0x7fffffff || K > 0x3fffffff) return 0;
+  return gemv_workspace_bytes(nullptr, bits, layout, M, N, K, false);
+}
+
+mpw_status mpw_qlinear_ws(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
+                          int64_t M, int64_t N, int64_t K, uint16_t* y, int path, void* workspace,
+                          size_t workspace_bytes, mpw_stream_t stream) {
+  return qlinear_impl(x, packed, scales, bits, layout, M, N, K, y, path, workspace, workspace_bytes, stream);
+}
+
+mpw_status mpw_qlinear_ex(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
+                          int64_t M, int64_t N, int64_t K, uint16_t* y, int path, mpw_stream_t stream) {
+  return qlinear_impl(x, packed, scales, bits, layout, M, N, K, y, path, nullptr, 0, stream);
 }
 
 mpw_status mpw_qlinear_path(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
@@ -199,8 +223,10 @@ mpw_status mpw_qlinear(const uint16_t* x, const uint8_t* packed, const float* sc
   return mpw_qlinear_ex(x, packed, scales, bits, MPW_LAYOUT_CANONICAL, M, N, K, y, MPW_PATH_AUTO, stream);
 }
 
-mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count, uint16_t* const* slots,
-                          int64_t num_slots, int64_t M, mpw_stream_t stream) {
+namespace {
+
+mpw_status recipe_check(const mpw_linear* layers, int64_t count, uint16_t* const* slots, int64_t num_slots,
+                        int64_t M) {
   if (layers == nullptr || slots == nullptr || count < 1 || num_slots < 1 || M < 1 || M > 32)
     return MPW_E_INVALID_ARG;
   for (int64_t i = 0; i < count; ++i) {
@@ -218,14 +244,49 @@ mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count, uint16_t* con
     if (!aligned(L.packed, 16) || !aligned(L.scales, 4)) return MPW_E_MISALIGNED;
     if (L.layout == MPW_LAYOUT_PAIRED && !aligned(slots[L.in_slot], 16)) return MPW_E_MISALIGNED;
   }
+  return MPW_OK;
+}
+
+size_t recipe_ws_bytes(const mpw_linear* layers, int64_t count, int64_t M) {
+  size_t b = 0;
+  for (int64_t i = 0; i < count; ++i) {
+    const mpw_linear& L = layers[i];
+    const size_t need = gemv_workspace_bytes(nullptr, L.bits, L.layout, M, L.N, L.K, L.norm_input != 0);
+    if (need > b) b = need;
+  }
+  return b;
+}
+
+}  // namespace
+
+size_t mpw_recipe_workspace_bytes(const mpw_linear* layers, int64_t count, int64_t M) {
+  if (layers == nullptr || count < 1 || M < 1 || M > 32) return 0;
+  for (int64_t i = 0; i < count; ++i)
+    if (!bits_ok(layers[i].bits) || !layout_ok(layers[i].layout) || layers[i].N < 1 || layers[i].K < 1) return 0;
+  return recipe_ws_bytes(layers, count, M);
+}
+
+mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count, uint16_t* const* slots, int64_t num_slots,
+                             int64_t M, void* workspace, size_t workspace_bytes, mpw_stream_t stream) {
+  const mpw_status st = recipe_check(layers, count, slots, num_slots, M);
+  if (st != MPW_OK) return st;
+  if (workspace != nullptr) {
+    if (!aligned(workspace, 16)) return MPW_E_MISALIGNED;
+    if (workspace_bytes < recipe_ws_bytes(layers, count, M)) return MPW_E_INVALID_ARG;
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   for (int64_t i = 0; i < count; ++i) {
     const mpw_linear& L = layers[i];
     cudaError_t e = launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, L.layout, M, L.N, L.K,
-                                slots[L.out_slot], L.norm_input != 0, s);
+                                slots[L.out_slot], L.norm_input != 0, workspace, workspace_bytes, s);
     if (e != cudaSuccess) return MPW_E_CUDA;
   }
   return MPW_OK;
+}
+
+mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count, uint16_t* const* slots,
+                          int64_t num_slots, int64_t M, mpw_stream_t stream) {
+  return mpw_recipe_run_ws(layers, count, slots, num_slots, M, nullptr, 0, stream);
 }
 
 mpw_status mpw_device_error(int32_t* code) {

@@ -439,12 +439,29 @@ cudaError_t gemv_bits(const uint16_t* x, int64_t M, const uint8_t* packed, const
 
 }  // namespace
 
+size_t gemv_workspace_bytes(const uint16_t* x_or_null, int bits, int layout, int64_t M, int64_t N, int64_t K,
+                            bool norm_input) {
+  const int64_t pass = norm_input ? 8 : 32;
+  const int64_t m1 = M < pass ? M : pass;
+  // alignment of x is the caller's business here: assume the kernel takes it
+  const uint16_t* xa = x_or_null != nullptr ? x_or_null : reinterpret_cast<const uint16_t*>(256);
+  if (!gemv_sk_supported(xa, m1, N, K, norm_input)) return 0;
+  size_t b = gemv_sk_workspace_bytes(bits, layout, m1, N, K, norm_input);
+  const int64_t last = M % pass;
+  if (M > pass && last != 0) {
+    const size_t b2 = gemv_sk_workspace_bytes(bits, layout, last, N, K, norm_input);
+    if (b2 > b) b = b2;
+  }
+  return b;
+}
+
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
                         int layout, int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm_input,
-                        cudaStream_t stream) {
+                        void* ws, size_t ws_bytes, cudaStream_t stream) {
   // Tensor-core decode kernels in passes of up to 32 tokens (8 with
-  // norm_input).  MPW_GEMV_KERNEL=mma selects the register-streaming variant
-  // for canonical rows (tuning aid).
+  // norm_input): the stream-K kernel when a workspace is given, else the
+  // per-tile TMA kernel.  MPW_GEMV_KERNEL=mma selects the register-streaming
+  // variant for canonical rows (tuning aid).
   static const bool use_mma = [] {
     const char* e = getenv("MPW_GEMV_KERNEL");
     return e != nullptr && e[0] == 'm';
@@ -452,15 +469,23 @@ cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* s
   const int64_t pass = norm_input ? 8 : 32;
   const int64_t m1 = M < pass ? M : pass;
   const bool paired = layout == kLayoutPaired;
+  const bool sk = ws != nullptr && !use_mma && gemv_sk_supported(x, m1, N, K, norm_input);
   const bool tma = (paired || !use_mma) && gemv_tma_supported(x, m1, N, K, norm_input);
   if (paired && !tma) return cudaErrorInvalidValue;
-  if (tma || gemv_mma_supported(m1, N, K, norm_input)) {
+  if (sk || tma || gemv_mma_supported(m1, N, K, norm_input)) {
     for (int64_t m0 = 0; m0 < M; m0 += pass) {
       const int64_t mt = M - m0 < pass ? M - m0 : pass;
-      cudaError_t e = tma ? launch_gemv_tma(x + m0 * K, packed, scales, bits, layout, mt, N, K, y + m0 * N,
-                                            norm_input, /*pdl=*/true, stream)
-                          : launch_gemv_mma(x + m0 * K, packed, scales, bits, mt, N, K, y + m0 * N, norm_input,
-                                            /*pdl=*/true, stream);
+      bool used = false;
+      cudaError_t e = cudaSuccess;
+      if (sk)
+        e = launch_gemv_sk(x + m0 * K, packed, scales, bits, layout, mt, N, K, y + m0 * N, norm_input, ws,
+                           ws_bytes, stream, &used);
+      if (e != cudaSuccess) return e;
+      if (!used)
+        e = tma ? launch_gemv_tma(x + m0 * K, packed, scales, bits, layout, mt, N, K, y + m0 * N, norm_input,
+                                  /*pdl=*/true, stream)
+                : launch_gemv_mma(x + m0 * K, packed, scales, bits, mt, N, K, y + m0 * N, norm_input,
+                                  /*pdl=*/true, stream);
       if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();

@@ -56,7 +56,10 @@ cudaError_t launch_repack(const uint8_t* in, int64_t N, int64_t K, int bits, uin
 // paired layout needs a shape the TMA kernel takes (checked by the caller).
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* scales,
                         int bits, int layout, int64_t M, int64_t N, int64_t K, uint16_t* y,
-                        bool norm_input, cudaStream_t stream);
+                        bool norm_input, void* ws, size_t ws_bytes, cudaStream_t stream);
+// Workspace bytes launch_gemv uses for these arguments (0 if none).
+size_t gemv_workspace_bytes(const uint16_t* x_or_null, int bits, int layout, int64_t M, int64_t N,
+                            int64_t K, bool norm_input);
 // The CUDA-core decode kernels alone (x in registers for K <= 17408, else x
 // staged in shared memory), in passes of two tokens.
 cudaError_t launch_gemv_cuda_core(const uint16_t* x, const uint8_t* packed, const float* scales,
@@ -77,6 +80,17 @@ bool gemv_tma_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, bool
 cudaError_t launch_gemv_tma(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
                             int layout, int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm,
                             bool pdl, cudaStream_t stream);
+
+// gemv_sk.cu: decode linear with the (tile, chunk) units split evenly over
+// a persistent grid; split tiles are combined in a caller workspace (zeroed
+// before its first use; the kernel leaves its counters at zero).  *used is
+// set when the kernel was launched; it is left false (and nothing launched)
+// when the workspace is missing or smaller than gemv_sk_workspace_bytes.
+bool gemv_sk_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, bool norm);
+size_t gemv_sk_workspace_bytes(int bits, int layout, int64_t M, int64_t N, int64_t K, bool norm);
+cudaError_t launch_gemv_sk(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
+                           int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, void* ws, size_t ws_bytes,
+                           cudaStream_t stream, bool* used);
 
 // gemm.cu: tcgen05 prefill GEMM; returns cudaErrorNotSupported for shapes it
 // does not take (the caller then uses the GEMV path).

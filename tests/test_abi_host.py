@@ -31,7 +31,8 @@ def test_header_declares_the_boundary():
     for want in ("mpw_quantize_pack", "mpw_unpack", "mpw_dequantize", "mpw_qlinear",
                  "mpw_qlinear_path", "mpw_recipe_run", "mpw_packed_row_bytes",
                  "mpw_status_str", "mpw_version", "mpw_device_error", "mpw_repack",
-                 "mpw_qlinear_ex"):
+                 "mpw_qlinear_ex", "mpw_qlinear_ws", "mpw_qlinear_workspace_bytes",
+                 "mpw_recipe_run_ws", "mpw_recipe_workspace_bytes"):
         assert want in names
 
 
@@ -126,6 +127,27 @@ def test_qlinear_ex_validation():
     assert L.mpw_qlinear_ex(A16 + 2, A16B, A16, 5, 1, 1, 4, 64, A16, 0, 0) == mpw.MPW_E_MISALIGNED
     assert L.mpw_qlinear_ex(A16, A16B, A16, 5, 1, 1, 4, 64, A16, 3, 0) == mpw.MPW_E_INVALID_ARG
     assert L.mpw_qlinear_ex(A16, A16B, A16, 2, 1, 1, 4, 64, A16, 0, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+
+
+def test_qlinear_ws_validation():
+    L = mpw.lib
+    # a workspace must be 16-byte aligned; argument errors come first
+    assert L.mpw_qlinear_ws(A16, A16B, A16, 5, 0, 1, 4, 64, A16, 0, A16 + 8, 4096, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_qlinear_ws(A16, A16B, A16, 3, 0, 1, 4, 64, A16, 0, A16, 4096, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    assert L.mpw_qlinear_ws(0, A16B, A16, 5, 0, 1, 4, 64, A16, 0, A16, 4096, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_workspace_bytes(3, 0, 1, 4, 64) == 0
+    assert L.mpw_qlinear_workspace_bytes(5, 2, 1, 4, 64) == 0
+    assert L.mpw_qlinear_workspace_bytes(5, 0, 33, 4, 64) == 0      # not a decode call
+
+
+def test_recipe_run_ws_validation():
+    L = mpw.lib
+    slots = (ctypes.c_void_p * 3)(A16, A16B, A16 + 0x100)
+    good = (A16, A16B, 8, 64, 6, 0, 1, 0)
+    assert L.mpw_recipe_run_ws(_layers(good), 1, slots, 3, 1, A16 + 4, 4096, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_recipe_run_ws(_layers(good), 0, slots, 3, 1, A16, 4096, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_recipe_workspace_bytes(_layers(good), 0, 1) == 0
+    assert L.mpw_recipe_workspace_bytes(_layers(good), 1, 33) == 0
 
 
 def _layers(*specs):
