@@ -5,7 +5,7 @@ This module only marshals arguments: it checks tensor dtypes, devices and
 shapes, allocates outputs with torch when the caller does not pass them, and
 forwards raw device pointers and the current CUDA stream.  Every step of the
 computation runs in the library's CUDA kernels; there is no CPU fallback, and
-importing the package fails if the library has not been built.
+the first call raises ImportError if the library has not been built.
 
 Build: ``python -m mixed_precision_weight_row_b200.build``.
 """
@@ -100,7 +100,20 @@ def _load():
     return L
 
 
-lib = _load()
+class _Lib:
+    """libmpw.so, opened on first use.  The build step imports this package
+    before the library exists, so the import itself does not open it; the
+    first call raises ImportError if the library has not been built."""
+
+    _handle = None
+
+    def __getattr__(self, name):
+        if _Lib._handle is None:
+            _Lib._handle = _load()
+        return getattr(_Lib._handle, name)
+
+
+lib = _Lib()
 
 
 def status_str(status: int) -> str:
