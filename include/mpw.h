@@ -64,7 +64,8 @@ typedef enum mpw_status {
   MPW_E_MISALIGNED = 3,       /* pointer alignment rule above violated */
   MPW_E_CUDA = 4,             /* a CUDA runtime call or launch failed */
   MPW_E_NONFINITE = 5,        /* reserved: reported through the flag word */
-  MPW_E_TIMEOUT = 6           /* a device-side wait gave up (see mpw_device_error) */
+  MPW_E_TIMEOUT = 6,          /* a device-side wait gave up (see mpw_device_error) */
+  MPW_E_SCRATCH_LIMIT = 7     /* mpw_qlinear_noalloc: the call needs more than its fixed scratch */
 } mpw_status;
 
 /* Static English text for a status code; never NULL. */
@@ -248,6 +249,35 @@ MPW_API size_t mpw_recipe_workspace_bytes(const mpw_linear* layers, int64_t coun
 MPW_API mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count,
                                      uint16_t* const* slots, int64_t num_slots, int64_t M,
                                      void* workspace, size_t workspace_bytes, mpw_stream_t stream);
+
+/*
+ * mpw_qlinear_noalloc -- the decode linear (M <= 32) on the stream-K kernel,
+ * with its workspace taken from a fixed array inside the library instead of
+ * from the caller, so that the call allocates no memory of any kind.
+ *
+ * No page describes this: it has no counterpart in the paper.  It exists for
+ * callers that must not allocate device memory at all -- code embedded in a
+ * host program that owns every allocation, work recorded where allocation
+ * calls are not allowed, or loops with a strict no-allocation rule -- and
+ * that therefore cannot provide the workspace mpw_qlinear_ws needs.
+ *   - The array holds MPW_NOALLOC_SCRATCH_BYTES (4 MiB) on every device that
+ *     loads the library, for the life of the process.  A call whose
+ *     workspace would exceed it returns MPW_E_SCRATCH_LIMIT and launches
+ *     nothing; mpw_qlinear_workspace_bytes tells the size in advance.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the array.  Each call clears the per-tile counters
+ *     it uses (a memset on `stream`) before its kernel; the partial sums need
+ *     no clearing.  Calls that overlap on the GPU (on different streams, or
+ *     in different host threads) race on the array and give wrong results.
+ *   - Arguments as mpw_qlinear_ex, with M in 1..32, K % 8 == 0 and x 16-byte
+ *     aligned (MPW_E_INVALID_ARG / MPW_E_MISALIGNED otherwise).
+ */
+#define MPW_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+MPW_API mpw_status mpw_qlinear_noalloc(const uint16_t* x, const uint8_t* packed, const float* scales,
+                                       int bits, int layout, int64_t M, int64_t N, int64_t K,
+                                       uint16_t* y, mpw_stream_t stream);
 
 /*
  * mpw_device_error -- synchronises the current device, returns in *code the

@@ -30,6 +30,7 @@ MPW_E_MISALIGNED = 3
 MPW_E_CUDA = 4
 MPW_E_NONFINITE = 5
 MPW_E_TIMEOUT = 6
+MPW_E_SCRATCH_LIMIT = 7
 
 PATHS = {"auto": 0, "gemv": 1, "gemm": 2}
 # Packed layouts (mpw_layout): the canonical stream and its paired-halves
@@ -93,6 +94,8 @@ def _load():
     L.mpw_recipe_run_ws.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp,
                                     ctypes.c_size_t, vp]
     L.mpw_recipe_run_ws.restype = c_int
+    L.mpw_qlinear_noalloc.argtypes = [vp, vp, vp, c_int, c_int, i64, i64, i64, vp, vp]
+    L.mpw_qlinear_noalloc.restype = c_int
     L.mpw_recipe_run.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp]
     L.mpw_recipe_run.restype = c_int
     L.mpw_device_error.argtypes = [ctypes.POINTER(i32)]

@@ -107,6 +107,7 @@ const char* mpw_status_str(int status) {
     case MPW_E_CUDA: return "CUDA error";
     case MPW_E_NONFINITE: return "non-finite input";
     case MPW_E_TIMEOUT: return "device-side wait timed out";
+    case MPW_E_SCRATCH_LIMIT: return "call needs more than the fixed scratch of mpw_qlinear_noalloc";
     default: return "unknown status";
   }
 }

@@ -41,6 +41,7 @@
 #include <type_traits>
 
 #include "expand.cuh"
+#include "mpw.h"
 #include "mpw_internal.h"
 #include "tc_ptx.cuh"
 
@@ -663,3 +664,64 @@ cudaError_t launch_gemv_sk(const uint16_t* x, const uint8_t* packed, const float
 }
 
 }  // namespace mpw
+
+// ---------------------------------------------------------------------------
+// mpw_qlinear_noalloc: the stream-K decode linear with its workspace in a
+// fixed device array, for callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------
+
+namespace mpw {
+
+// Zero-initialised when the library is loaded; every device holds a copy.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MPW_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of the array on the current device, looked up once per
+// device (with that device current).  nullptr if the lookup failed.
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+}  // namespace mpw
+
+extern "C" MPW_API mpw_status mpw_qlinear_noalloc(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                                          int layout, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                          mpw_stream_t stream) {
+  using namespace mpw;
+  auto misaligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) != 0; };
+  if (bits < kMinBits || bits > kMaxBits) return MPW_E_UNSUPPORTED_BITS;
+  if (x == nullptr || packed == nullptr || scales == nullptr || y == nullptr) return MPW_E_INVALID_ARG;
+  if (M < 1 || M > 32 || N < 1 || K < 1 || N > 0x7fffffff || K > 0x3fffffff) return MPW_E_INVALID_ARG;
+  if (layout != kLayoutCanonical && layout != kLayoutPaired) return MPW_E_INVALID_ARG;
+  if (layout == kLayoutPaired && K % 32 != 0) return MPW_E_INVALID_ARG;
+  if (misaligned(packed, 16) || misaligned(x, 16) || misaligned(y, 2) || misaligned(scales, 4))
+    return MPW_E_MISALIGNED;
+  if (!gemv_sk_supported(x, M, N, K, false)) return MPW_E_INVALID_ARG;
+  const size_t need = gemv_sk_workspace_bytes(bits, layout, M, N, K, false);
+  if (need == 0 || need > MPW_NOALLOC_SCRATCH_BYTES) return MPW_E_SCRATCH_LIMIT;
+  void* ws = noalloc_scratch();
+  if (ws == nullptr) return MPW_E_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the counters of the call's tiles (first in the workspace) must start at zero
+  const size_t counter_bytes = static_cast<size_t>((N + 15) / 16) * 4;
+  if (cudaMemsetAsync(ws, 0, counter_bytes, s) != cudaSuccess) return MPW_E_CUDA;
+  bool used = false;
+  const cudaError_t e = launch_gemv_sk(x, packed, scales, bits, layout, M, N, K, y, false, ws,
+                                       MPW_NOALLOC_SCRATCH_BYTES, s, &used);
+  if (e != cudaSuccess || !used) return MPW_E_CUDA;
+  return MPW_OK;
+}
