@@ -232,7 +232,10 @@ typedef struct mpw_linear {
 /*
  * mpw_recipe_run -- apply a per-matrix bit-width recipe to a stack of linears:
  * launches `count` qlinear kernels in order on `stream` (capturable in a CUDA
- * graph).  slots[i] are device bf16 buffers; each must hold M * (largest N or
+ * graph).  Consecutive linears that read the same slot and write distinct
+ * other slots (q, k, v; gate, up) are independent: they run at the same time
+ * on library-internal streams of the device, forked from and joined back into
+ * `stream` by events, so the call stays ordered on `stream` as a whole.  slots[i] are device bf16 buffers; each must hold M * (largest N or
  * K that touches it) elements.  M must be in 1..32 (the decode pass).
  * A linear whose in_slot equals its out_slot is rejected.
  */
@@ -245,7 +248,7 @@ MPW_API mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count,
 MPW_API size_t mpw_recipe_workspace_bytes(const mpw_linear* layers, int64_t count, int64_t M);
 
 /* mpw_recipe_run with a decode workspace (see mpw_qlinear_workspace_bytes);
- * the linears run one after another and share it. */
+ * the linears run one after another (never side by side) and share it. */
 MPW_API mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count,
                                      uint16_t* const* slots, int64_t num_slots, int64_t M,
                                      void* workspace, size_t workspace_bytes, mpw_stream_t stream);

@@ -248,6 +248,56 @@ mpw_status recipe_check(const mpw_linear* layers, int64_t count, uint16_t* const
   return MPW_OK;
 }
 
+// ---- independent linears of a recipe run side by side ----
+// Consecutive linears that read the same slot and write distinct other slots
+// (q, k, v of a layer; gate and up) do not depend on one another.  The first
+// runs on the caller's stream, the others on library-internal streams of
+// the device, forked from and joined back into the caller's stream with
+// events, so that small matrices overlap large ones and one dependency
+// round-trip serves the group.
+constexpr int kMaxBranches = 4;
+
+struct Branches {
+  int device = -1;
+  bool ok = false;
+  cudaStream_t side[kMaxBranches - 1] = {};
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join[kMaxBranches - 1] = {};
+};
+Branches g_branches[kMaxDevices];
+std::mutex g_branch_mutex;
+
+// The current device's internal streams and events, created on first use;
+// nullptr if they could not be created (linears then run one by one).
+Branches* branches() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_branch_mutex);
+  Branches& br = g_branches[dev];
+  if (br.device != dev) {
+    bool ok = cudaEventCreateWithFlags(&br.fork, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < kMaxBranches - 1; ++i) {
+      ok = ok && cudaStreamCreateWithFlags(&br.side[i], cudaStreamNonBlocking) == cudaSuccess;
+      ok = ok && cudaEventCreateWithFlags(&br.join[i], cudaEventDisableTiming) == cudaSuccess;
+    }
+    br.ok = ok;
+    br.device = dev;
+  }
+  return br.ok ? &br : nullptr;
+}
+
+// End of the group of independent linears that starts at i.
+int64_t group_end(const mpw_linear* L, int64_t i, int64_t count) {
+  int64_t j = i + 1;
+  while (j < count && j - i < kMaxBranches && L[j].in_slot == L[i].in_slot) {
+    bool clash = false;
+    for (int64_t a = i; a < j; ++a) clash = clash || L[a].out_slot == L[j].out_slot;
+    if (clash) break;
+    ++j;
+  }
+  return j;
+}
+
 size_t recipe_ws_bytes(const mpw_linear* layers, int64_t count, int64_t M) {
   size_t b = 0;
   for (int64_t i = 0; i < count; ++i) {
@@ -276,11 +326,31 @@ mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count, uint16_t* 
     if (workspace_bytes < recipe_ws_bytes(layers, count, M)) return MPW_E_INVALID_ARG;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  for (int64_t i = 0; i < count; ++i) {
+  auto run = [&](int64_t i, cudaStream_t st) {
     const mpw_linear& L = layers[i];
-    cudaError_t e = launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, L.layout, M, L.N, L.K,
-                                slots[L.out_slot], L.norm_input != 0, workspace, workspace_bytes, s);
-    if (e != cudaSuccess) return MPW_E_CUDA;
+    return launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, L.layout, M, L.N, L.K, slots[L.out_slot],
+                       L.norm_input != 0, workspace, workspace_bytes, st);
+  };
+  // a shared workspace cannot serve linears that run at the same time
+  Branches* br = workspace == nullptr ? branches() : nullptr;
+  for (int64_t i = 0; i < count;) {
+    const int64_t j = br != nullptr ? group_end(layers, i, count) : i + 1;
+    if (j - i == 1) {
+      if (run(i, s) != cudaSuccess) return MPW_E_CUDA;
+      i = j;
+      continue;
+    }
+    if (cudaEventRecord(br->fork, s) != cudaSuccess) return MPW_E_CUDA;
+    for (int64_t k = 1; k < j - i; ++k) {
+      cudaStream_t side = br->side[k - 1];
+      if (cudaStreamWaitEvent(side, br->fork, 0) != cudaSuccess) return MPW_E_CUDA;
+      if (run(i + k, side) != cudaSuccess) return MPW_E_CUDA;
+      if (cudaEventRecord(br->join[k - 1], side) != cudaSuccess) return MPW_E_CUDA;
+    }
+    if (run(i, s) != cudaSuccess) return MPW_E_CUDA;
+    for (int64_t k = 1; k < j - i; ++k)
+      if (cudaStreamWaitEvent(s, br->join[k - 1], 0) != cudaSuccess) return MPW_E_CUDA;
+    i = j;
   }
   return MPW_OK;
 }
