@@ -8,13 +8,12 @@
 //
 // One CTA computes a 128-row (W) x 256-token (x) tile of y^T with
 // tcgen05.mma.cta_group::1.kind::f16, M=128, N=256, K=16:
-//   * Packed weights move in blocks of 128 codes (16*B bytes per row): warp 3
-//     copies them with 16-byte cp.async (consecutive lanes take consecutive
-//     16-byte units of a row, so each warp instruction reads whole lines)
-//     into a shared-memory ring whose row pitch is padded to an odd number
-//     of 16-byte units, so the converters' 16-byte reads are free of bank
-//     conflicts; completion reaches an mbarrier through
-//     cp.async.mbarrier.arrive.
+//   * Packed weights move in blocks of 128 codes (16*B bytes per row), one 2D
+//     TMA per block ({16*B bytes x 128 rows}) into a 3-stage ring; rows past
+//     N and bytes past the row read as zeros.  The converters read a row's
+//     16-byte units; for b = 4 and b = 8 the TMA's 64- and 128-byte swizzle
+//     spreads eight consecutive rows over all banks, odd b are conflict-free
+//     as they are, and the other even b cost two to four ways.
 //   * A = 128 weight rows x 16 codes, held in TENSOR MEMORY.  Converter warps
 //     (two groups of four, alternating weight blocks; one row per thread)
 //     expand each pair of codes to an exact bf16x2 value with a bit-field
@@ -63,28 +62,25 @@ struct GemmCode {
   static constexpr int P = GemmParts<B>::parts;              // MMAs per k-step
   static constexpr uint32_t ACOLS = 64u * P;                 // tensor-memory columns per A stage
   static constexpr int SA = static_cast<int>((kTmemCols - kAccCols) / ACOLS);
-  // row pitch of a weight stage: 16*B bytes padded to an odd number of
-  // 16-byte units
-  static constexpr uint32_t PITCH = 16u * (B % 2 == 1 ? B : B + 1);
+  // a weight stage is the TMA box: 128 rows of 16*B bytes
+  static constexpr uint32_t PITCH = 16u * B;
   static constexpr uint32_t WSTAGE = BM * PITCH;
+  static constexpr CUtensorMapSwizzle WSWZ =
+      B == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : (B == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE);
+  // byte offset of 16-byte unit u of row r inside a weight stage
+  static __device__ __forceinline__ uint32_t unit(int r, int u) {
+    if constexpr (B == 8) return r * 128u + 16u * (static_cast<uint32_t>(u) ^ (r & 7));
+    else if constexpr (B == 4) return r * 64u + 16u * (static_cast<uint32_t>(u) ^ ((r >> 1) & 3));
+    else return r * PITCH + 16u * u;
+  }
   static constexpr size_t SMEM = SX * kXStageBytes + SW * WSTAGE + 1024 /*align*/ + 256 /*barriers*/;
   static_assert(SMEM <= 232448, "shared memory per block");
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src))
-               : "memory");
-}
-
-// Arrives on the mbarrier once every cp.async this thread issued has landed
-// (the arrival is counted in the barrier's expected count).
-__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
 
 template <int B, bool PAIRED>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restrict__ packed,
+gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
             const float* __restrict__ scales, uint16_t* __restrict__ y, int M, int N, int K, int rb,
             int32_t* err) {
   using C = GemmCode<B>;
@@ -120,7 +116,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restric
       ptx::mbar_init(empty_x(s), 1);
     }
     for (int s = 0; s < SW; ++s) {
-      ptx::mbar_init(full_w(s), 32);        // the weight producer's lanes
+      ptx::mbar_init(full_w(s), 1);
       ptx::mbar_init(empty_w(s), 128);      // one converter group
     }
     for (int s = 0; s < SA; ++s) {
@@ -130,6 +126,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restric
     ptx::mbar_init(acc_full, 1);
     ptx::mbar_fence_init();
     ptx::prefetch_tmap(&tmap_x);
+    ptx::prefetch_tmap(&tmap_w);
   }
   if (warp == 2) {
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
@@ -157,33 +154,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restric
       for (int kb = max(0, issued - SX); kb < issued; ++kb) ptx::mbar_wait(full_x(kb % SX), (kb / SX) & 1, err);
     }
   } else if (warp == 3) {
-    // ---------------- weight producer: 16-byte cp.async ----------------
-    int issued = 0;
-    for (int wb = 0; wb < WBs; ++wb) {
-      const int s = wb % SW;
-      bool ok = true;
-      if (lane == 0) ok = ptx::mbar_wait(empty_w(s), ((wb / SW) & 1) ^ 1, err);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      // the last block of a row may be shorter (the row ends at rb bytes)
-      const int units = min(B, (rb - wb * 16 * B) / 16);
-      const uint8_t* blk = packed + static_cast<size_t>(wb) * 16 * B;
-      const uint32_t dst0 = ws0 + s * C::WSTAGE;
-#pragma unroll 4
-      for (int idx = lane; idx < BM * B; idx += 32) {
-        const int r = idx / B, u = idx - r * B;
-        if (u < units) {
-          const int n = min(n0 + r, N - 1);   // rows past N: any valid row (their outputs are not stored)
-          cp_async16(dst0 + r * C::PITCH + u * 16, blk + static_cast<size_t>(n) * rb + u * 16);
-        }
+    // ---------------- weight producer: one TMA per block ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int wb = 0; wb < WBs; ++wb) {
+        const int s = wb % SW;
+        if (!ptx::mbar_wait(empty_w(s), ((wb / SW) & 1) ^ 1, err)) break;
+        ptx::mbar_arrive_expect_tx(full_w(s), C::WSTAGE);
+        ptx::tma_load_2d(ws0 + s * C::WSTAGE, &tmap_w, full_w(s), wb * 16 * B, n0);
+        issued = wb + 1;
       }
-      cp_async_arrive(full_w(s));
-      issued = wb + 1;
-    }
-    // nothing may still be landing in shared memory when the CTA exits
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    if (lane == 0)
+      // nothing may still be landing in shared memory when the CTA exits
       for (int wb = max(0, issued - SW); wb < issued; ++wb) ptx::mbar_wait(full_w(wb % SW), (wb / SW) & 1, err);
+    }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -224,10 +207,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint8_t* __restric
       if (!ok) break;
       // the row's 4 groups: 16*B bytes, read as 16-byte units
       uint32_t w[4 * B + 1];
-      const uint4* src = reinterpret_cast<const uint4*>(gsmem + SX * kXStageBytes + ws * C::WSTAGE + r * C::PITCH);
+      const uint8_t* stage = gsmem + SX * kXStageBytes + ws * C::WSTAGE;
 #pragma unroll
       for (int i = 0; i < B; ++i) {
-        const uint4 v = src[i];
+        const uint4 v = *reinterpret_cast<const uint4*>(stage + C::unit(r, i));
         w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
       }
       w[4 * B] = 0u;
@@ -298,13 +281,23 @@ cudaError_t run_gemm(const uint16_t* x, const uint8_t* packed, const float* scal
                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  const int64_t rb = 16 * ((K * B + 127) / 128);
+  CUtensorMap tmap_w;
+  {
+    const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(N)};
+    const cuuint64_t wstrides[1] = {static_cast<cuuint64_t>(rb)};
+    const cuuint32_t wbox[2] = {static_cast<cuuint32_t>(16 * B), static_cast<cuuint32_t>(BM)};
+    if (encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), wdims, wstrides, wbox,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, C::WSWZ, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   auto kern = gemm_kernel<B, PAIRED>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>((N + BM - 1) / BM), static_cast<unsigned>((M + BN - 1) / BN));
-  kern<<<grid, kThreads, C::SMEM, stream>>>(tmap, packed, scales, y, static_cast<int>(M), static_cast<int>(N),
-                                            static_cast<int>(K), static_cast<int>(16 * ((K * B + 127) / 128)),
-                                            err);
+  kern<<<grid, kThreads, C::SMEM, stream>>>(tmap, tmap_w, scales, y, static_cast<int>(M), static_cast<int>(N),
+                                            static_cast<int>(K), static_cast<int>(rb), err);
   return cudaGetLastError();
 }
 

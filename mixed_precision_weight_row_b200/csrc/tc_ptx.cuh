@@ -72,8 +72,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 16; ++i)
-      if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    for (int i = 0; i < 128; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer() - t0 > limit_ns) {
       if (err != nullptr) atomicExch(err, 1);
       return false;
