@@ -466,6 +466,25 @@ cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* s
     const char* e = getenv("MPW_GEMV_KERNEL");
     return e != nullptr && e[0] == 'm';
   }();
+  static const bool use_tc = [] {
+    const char* e = getenv("MPW_GEMV_KERNEL");
+    return e != nullptr && e[0] == 't' && e[1] == 'c';
+  }();
+  // Tensor-memory kernel (passes of 32 tokens) where it is the faster one
+  // (MPW_GEMV_KERNEL=tc forces it, a tuning aid).
+  {
+    const int64_t m1 = M < 32 ? M : 32;
+    if (ws == nullptr && !use_mma && gemv_tc_supported(x, m1, N, K, norm_input) &&
+        (use_tc || gemv_tc_preferred(bits, m1, N, K))) {
+      for (int64_t m0 = 0; m0 < M; m0 += 32) {
+        const int64_t mt = M - m0 < 32 ? M - m0 : 32;
+        cudaError_t e = launch_gemv_tc(x + m0 * K, packed, scales, bits, layout, mt, N, K, y + m0 * N, norm_input,
+                                       stream);
+        if (e != cudaSuccess) return e;
+      }
+      return cudaGetLastError();
+    }
+  }
   const int64_t pass = norm_input ? 8 : 32;
   const int64_t m1 = M < pass ? M : pass;
   const bool paired = layout == kLayoutPaired;

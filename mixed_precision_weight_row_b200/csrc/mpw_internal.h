@@ -92,6 +92,15 @@ cudaError_t launch_gemv_sk(const uint16_t* x, const uint8_t* packed, const float
                            int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, void* ws, size_t ws_bytes,
                            cudaStream_t stream, bool* used);
 
+// gemv_tc.cu: decode linear for M <= 32 on tcgen05 tensor cores (weights
+// expanded into tensor memory, 128-row tiles, K split over a cluster when
+// there are few tiles).
+bool gemv_tc_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, bool norm);
+// Whether the shape is one where this kernel beats the per-tile decode kernel.
+bool gemv_tc_preferred(int bits, int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemv_tc(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
+                           int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, cudaStream_t stream);
+
 // gemm.cu: tcgen05 prefill GEMM; returns cudaErrorNotSupported for shapes it
 // does not take (the caller then uses the GEMV path).
 cudaError_t launch_gemm(const uint16_t* x, const uint8_t* packed, const float* scales,
