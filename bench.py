@@ -233,7 +233,11 @@ def decode_setup(mpw, W_gpu, b, l2_bytes, layout="canonical"):
     return Pool(packed, scales, 4 * l2_bytes)
 
 
-def measure_decode(mpw, pool, b, M, K, N, steps, warmup, world=1, x=None, layout="canonical"):
+def measure_decode(mpw, pool, b, M, K, N, steps, warmup, world=1, x=None, layout="canonical", x_ready=True):
+    """Back-to-back launches over the pool's distinct matrices with one x.
+    No launch writes x, which each call states (x_ready) unless asked not to,
+    so that a launch's product may overlap its predecessor; x_ready=False
+    times the same launches as a dependent chain."""
     import torch
 
     import workloads as wl
@@ -244,7 +248,7 @@ def measure_decode(mpw, pool, b, M, K, N, steps, warmup, world=1, x=None, layout
 
     def step():
         for i in range(pool.P):
-            mpw.qlinear(x, pool.packed[i], pool.scales[i], b, y=y, layout=layout)
+            mpw.qlinear(x, pool.packed[i], pool.scales[i], b, y=y, layout=layout, x_ready=x_ready)
 
     g = graph_of(step)
     ms = time_graph(g, steps, warmup, world)
@@ -561,8 +565,9 @@ def main(argv=None):
     y1 = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
 
     def step():
+        # distinct matrices applied to one x: no launch writes x (x_ready)
         for i in range(pool.P):
-            mpw.qlinear(x1, pool.packed[i], pool.scales[i], HEADLINE_BITS, y=y1, layout=lay)
+            mpw.qlinear(x1, pool.packed[i], pool.scales[i], HEADLINE_BITS, y=y1, layout=lay, x_ready=True)
 
     g = graph_of(step)
     with ClockSampler(uuid) as cs:
@@ -578,6 +583,14 @@ def main(argv=None):
     achieved = alg_bytes / (us_launch * 1e-6) / 1e9
 
     extras = {}
+    if rank == 0:
+        # the same launches, each one waiting for its predecessor before it
+        # reads x (what a chain of dependent linears sees)
+        r = measure_decode(mpw, pool, HEADLINE_BITS, 1, K, N, max(20, args.steps // 4), 3, layout=lay,
+                           x=x1, x_ready=False)
+        extras["dependent_chain"] = {"us_per_launch": round(r["us_per_launch"], 4),
+                                     "weight_GBps": round(r["weight_GBps"], 1),
+                                     "pct_hbm": round(100.0 * r["alg_GBps"] / pk["hbm_gbs"], 2)}
     if rank == 0 and not args.quick:
         sweep = []
         for b in DECODE_BITS:

@@ -202,6 +202,31 @@ MPW_API mpw_status mpw_qlinear_ws(const uint16_t* x, const uint8_t* packed, cons
                                   mpw_stream_t stream);
 
 /*
+ * mpw_qlinear_flags -- mpw_qlinear_ex with flags (0 or MPW_QLINEAR_X_READY;
+ * other bits are MPW_E_INVALID_ARG).
+ *   MPW_QLINEAR_X_READY: the caller states that x was written before the
+ *   launch that precedes the current run of flagged calls on `stream` (the
+ *   consecutive calls made with this flag, this one included): neither a
+ *   call of the run nor the launch just before it wrote x.  Typical uses: q
+ *   called without the flag, then k and v with it, all three reading a hidden
+ *   state written earlier; a set of matrices applied to one x that was
+ *   complete before the set began.  A flagged decode kernel lets the next
+ *   kernel start at once and loads x together with its weights without
+ *   waiting for its predecessor, so consecutive flagged calls overlap in
+ *   full; only its write of y waits for the preceding launch, so results
+ *   land in call order.  The statement suffices because this library's
+ *   unflagged decode kernels let their successor start only after they have
+ *   themselves waited for their predecessor; the launch before the run must
+ *   be one of this library's kernels, a copy, or a kernel launched without
+ *   programmatic dependent launch.  A false statement is a data race (stale
+ *   x), not an error code.  Results are those of mpw_qlinear_ex.
+ */
+#define MPW_QLINEAR_X_READY 1u
+MPW_API mpw_status mpw_qlinear_flags(const uint16_t* x, const uint8_t* packed, const float* scales,
+                                     int bits, int layout, int64_t M, int64_t N, int64_t K,
+                                     uint16_t* y, int path, unsigned flags, mpw_stream_t stream);
+
+/*
  * One linear of a recipe stack (DynaQuant "Step 3": every matrix carries its
  * own bit width).  Activations move between caller-owned "slots".
  *   packed, scales, N, K, bits  the quantized matrix (device pointers).
@@ -232,10 +257,11 @@ typedef struct mpw_linear {
 /*
  * mpw_recipe_run -- apply a per-matrix bit-width recipe to a stack of linears:
  * launches `count` qlinear kernels in order on `stream` (capturable in a CUDA
- * graph).  Consecutive linears that read the same slot and write distinct
- * other slots (q, k, v; gate, up) are independent: they run at the same time
- * on library-internal streams of the device, forked from and joined back into
- * `stream` by events, so the call stays ordered on `stream` as a whole.  slots[i] are device bf16 buffers; each must hold M * (largest N or
+ * graph).  A linear whose input bytes were written neither by the linear
+ * before the current run of such linears nor by one inside it (k and v after
+ * q; up after gate) is launched with MPW_QLINEAR_X_READY, so that it runs
+ * alongside its predecessors; the first linear never is.  Outputs land in
+ * order.  slots[i] are device bf16 buffers; each must hold M * (largest N or
  * K that touches it) elements.  M must be in 1..32 (the decode pass).
  * A linear whose in_slot equals its out_slot is rejected.
  */
@@ -248,7 +274,7 @@ MPW_API mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count,
 MPW_API size_t mpw_recipe_workspace_bytes(const mpw_linear* layers, int64_t count, int64_t M);
 
 /* mpw_recipe_run with a decode workspace (see mpw_qlinear_workspace_bytes);
- * the linears run one after another (never side by side) and share it. */
+ * the linears that use it run one after another and share it. */
 MPW_API mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count,
                                      uint16_t* const* slots, int64_t num_slots, int64_t M,
                                      void* workspace, size_t workspace_bytes, mpw_stream_t stream);

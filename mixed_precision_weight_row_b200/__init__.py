@@ -36,6 +36,9 @@ PATHS = {"auto": 0, "gemv": 1, "gemm": 2}
 # Packed layouts (mpw_layout): the canonical stream and its paired-halves
 # re-ordering, which the decode kernels read fastest (K % 32 == 0).
 LAYOUTS = {"canonical": 0, "paired": 1}
+# mpw_qlinear_flags: x was written before the launch preceding the run of
+# flagged calls
+X_READY = 1
 
 
 class MPWError(RuntimeError):
@@ -89,6 +92,8 @@ def _load():
     L.mpw_qlinear_workspace_bytes.restype = ctypes.c_size_t
     L.mpw_qlinear_ws.argtypes = [vp, vp, vp, c_int, c_int, i64, i64, i64, vp, c_int, vp, ctypes.c_size_t, vp]
     L.mpw_qlinear_ws.restype = c_int
+    L.mpw_qlinear_flags.argtypes = [vp, vp, vp, c_int, c_int, i64, i64, i64, vp, c_int, ctypes.c_uint, vp]
+    L.mpw_qlinear_flags.restype = c_int
     L.mpw_recipe_workspace_bytes.argtypes = [ctypes.POINTER(_Linear), i64, i64]
     L.mpw_recipe_workspace_bytes.restype = ctypes.c_size_t
     L.mpw_recipe_run_ws.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp,
@@ -251,14 +256,19 @@ def repack(packed, K: int, bits: int, layout_in: str = "canonical", layout_out: 
 
 
 def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: str = "canonical",
-            stream=None, use_workspace: bool = False):
+            stream=None, use_workspace: bool = False, x_ready: bool = False):
     """y = x @ (q * s)^T with x bf16 [M, K]; returns y bf16 [M, N].
 
     With ``use_workspace`` the decode path (M <= 32) gets this stream's
     workspace and runs the stream-K kernel; without it (the default, faster
-    on every measured shape) the per-tile kernel."""
+    on every measured shape) the per-tile kernel.  ``x_ready`` states that x
+    was written before the launch that precedes the current run of x_ready
+    calls on the stream (MPW_QLINEAR_X_READY in mpw.h); it cannot be combined
+    with a workspace."""
     import torch
 
+    if x_ready and use_workspace:
+        raise ValueError("x_ready cannot be combined with use_workspace")
     _need(x, torch.bfloat16, "x", 2)
     _need(packed, torch.uint8, "packed", 2)
     _need(scales, torch.float32, "scales", 1)
@@ -271,6 +281,11 @@ def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: st
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     _need(y, torch.bfloat16, "y")
+    if x_ready:
+        _check(lib.mpw_qlinear_flags(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits),
+                                     LAYOUTS[layout], M, N, K, y.data_ptr(), PATHS[path], X_READY,
+                                     _stream(stream)), "mpw_qlinear_flags")
+        return y
     ws, ws_bytes = None, 0
     if use_workspace:
         need = qlinear_workspace_bytes(bits, min(M, 32), N, K, layout) if M <= 32 or path == "gemv" else 0

@@ -172,8 +172,9 @@ namespace {
 
 mpw_status qlinear_impl(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
                         int64_t M, int64_t N, int64_t K, uint16_t* y, int path, void* ws, size_t ws_bytes,
-                        mpw_stream_t stream) {
+                        unsigned flags, mpw_stream_t stream) {
   if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
+  if ((flags & ~static_cast<unsigned>(MPW_QLINEAR_X_READY)) != 0) return MPW_E_INVALID_ARG;
   if (x == nullptr || packed == nullptr || scales == nullptr || y == nullptr || M < 1 || N < 1 ||
       K < 1)
     return MPW_E_INVALID_ARG;
@@ -191,7 +192,8 @@ mpw_status qlinear_impl(const uint16_t* x, const uint8_t* packed, const float* s
   }
   if (path == MPW_PATH_GEMM) return MPW_E_INVALID_ARG;  // shape the GEMM does not take
   if (ws != nullptr && ws_bytes < gemv_workspace_bytes(x, bits, layout, M, N, K, false)) return MPW_E_INVALID_ARG;
-  return from_cuda(launch_gemv(x, packed, scales, bits, layout, M, N, K, y, false, ws, ws_bytes, s));
+  return from_cuda(launch_gemv(x, packed, scales, bits, layout, M, N, K, y, false, ws, ws_bytes, s,
+                               (flags & MPW_QLINEAR_X_READY) != 0));
 }
 
 }  // namespace
@@ -205,12 +207,18 @@ size_t mpw_qlinear_workspace_bytes(int bits, int layout, int64_t M, int64_t N, i
 mpw_status mpw_qlinear_ws(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
                           int64_t M, int64_t N, int64_t K, uint16_t* y, int path, void* workspace,
                           size_t workspace_bytes, mpw_stream_t stream) {
-  return qlinear_impl(x, packed, scales, bits, layout, M, N, K, y, path, workspace, workspace_bytes, stream);
+  return qlinear_impl(x, packed, scales, bits, layout, M, N, K, y, path, workspace, workspace_bytes, 0u, stream);
+}
+
+mpw_status mpw_qlinear_flags(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
+                             int64_t M, int64_t N, int64_t K, uint16_t* y, int path, unsigned flags,
+                             mpw_stream_t stream) {
+  return qlinear_impl(x, packed, scales, bits, layout, M, N, K, y, path, nullptr, 0, flags, stream);
 }
 
 mpw_status mpw_qlinear_ex(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
                           int64_t M, int64_t N, int64_t K, uint16_t* y, int path, mpw_stream_t stream) {
-  return qlinear_impl(x, packed, scales, bits, layout, M, N, K, y, path, nullptr, 0, stream);
+  return qlinear_impl(x, packed, scales, bits, layout, M, N, K, y, path, nullptr, 0, 0u, stream);
 }
 
 mpw_status mpw_qlinear_path(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
@@ -248,56 +256,6 @@ mpw_status recipe_check(const mpw_linear* layers, int64_t count, uint16_t* const
   return MPW_OK;
 }
 
-// ---- independent linears of a recipe run side by side ----
-// Consecutive linears that read the same slot and write distinct other slots
-// (q, k, v of a layer; gate and up) do not depend on one another.  The first
-// runs on the caller's stream, the others on library-internal streams of
-// the device, forked from and joined back into the caller's stream with
-// events, so that small matrices overlap large ones and one dependency
-// round-trip serves the group.
-constexpr int kMaxBranches = 4;
-
-struct Branches {
-  int device = -1;
-  bool ok = false;
-  cudaStream_t side[kMaxBranches - 1] = {};
-  cudaEvent_t fork = nullptr;
-  cudaEvent_t join[kMaxBranches - 1] = {};
-};
-Branches g_branches[kMaxDevices];
-std::mutex g_branch_mutex;
-
-// The current device's internal streams and events, created on first use;
-// nullptr if they could not be created (linears then run one by one).
-Branches* branches() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_branch_mutex);
-  Branches& br = g_branches[dev];
-  if (br.device != dev) {
-    bool ok = cudaEventCreateWithFlags(&br.fork, cudaEventDisableTiming) == cudaSuccess;
-    for (int i = 0; i < kMaxBranches - 1; ++i) {
-      ok = ok && cudaStreamCreateWithFlags(&br.side[i], cudaStreamNonBlocking) == cudaSuccess;
-      ok = ok && cudaEventCreateWithFlags(&br.join[i], cudaEventDisableTiming) == cudaSuccess;
-    }
-    br.ok = ok;
-    br.device = dev;
-  }
-  return br.ok ? &br : nullptr;
-}
-
-// End of the group of independent linears that starts at i.
-int64_t group_end(const mpw_linear* L, int64_t i, int64_t count) {
-  int64_t j = i + 1;
-  while (j < count && j - i < kMaxBranches && L[j].in_slot == L[i].in_slot) {
-    bool clash = false;
-    for (int64_t a = i; a < j; ++a) clash = clash || L[a].out_slot == L[j].out_slot;
-    if (clash) break;
-    ++j;
-  }
-  return j;
-}
-
 size_t recipe_ws_bytes(const mpw_linear* layers, int64_t count, int64_t M) {
   size_t b = 0;
   for (int64_t i = 0; i < count; ++i) {
@@ -326,31 +284,32 @@ mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count, uint16_t* 
     if (workspace_bytes < recipe_ws_bytes(layers, count, M)) return MPW_E_INVALID_ARG;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  auto run = [&](int64_t i, cudaStream_t st) {
+  auto run = [&](int64_t i, cudaStream_t st, bool x_ready) {
     const mpw_linear& L = layers[i];
     return launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, L.layout, M, L.N, L.K, slots[L.out_slot],
-                       L.norm_input != 0, workspace, workspace_bytes, st);
+                       L.norm_input != 0, workspace, workspace_bytes, st, x_ready);
   };
-  // a shared workspace cannot serve linears that run at the same time
-  Branches* br = workspace == nullptr ? branches() : nullptr;
-  for (int64_t i = 0; i < count;) {
-    const int64_t j = br != nullptr ? group_end(layers, i, count) : i + 1;
-    if (j - i == 1) {
-      if (run(i, s) != cudaSuccess) return MPW_E_CUDA;
-      i = j;
-      continue;
-    }
-    if (cudaEventRecord(br->fork, s) != cudaSuccess) return MPW_E_CUDA;
-    for (int64_t k = 1; k < j - i; ++k) {
-      cudaStream_t side = br->side[k - 1];
-      if (cudaStreamWaitEvent(side, br->fork, 0) != cudaSuccess) return MPW_E_CUDA;
-      if (run(i + k, side) != cudaSuccess) return MPW_E_CUDA;
-      if (cudaEventRecord(br->join[k - 1], side) != cudaSuccess) return MPW_E_CUDA;
-    }
-    if (run(i, s) != cudaSuccess) return MPW_E_CUDA;
-    for (int64_t k = 1; k < j - i; ++k)
-      if (cudaStreamWaitEvent(s, br->join[k - 1], 0) != cudaSuccess) return MPW_E_CUDA;
-    i = j;
+  // A linear whose input was written neither by the linear before the
+  // current run of x-ready linears nor by one inside it joins the run
+  // (MPW_QLINEAR_X_READY): k and v after q, up after gate.  Inputs and
+  // outputs are compared as byte ranges, so slots that alias are safe.  The
+  // first linear follows whatever the caller launched before: never.
+  constexpr int kRunMax = 8;
+  uintptr_t run_lo[kRunMax], run_hi[kRunMax];  // outputs of the run and of the linear before it
+  int nrun = 0;
+  for (int64_t i = 0; i < count; ++i) {
+    const mpw_linear& L = layers[i];
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(slots[L.in_slot]);
+    const uintptr_t xb = xa + static_cast<uintptr_t>(M * L.K) * 2u;
+    const uintptr_t ya = reinterpret_cast<uintptr_t>(slots[L.out_slot]);
+    const uintptr_t yb = ya + static_cast<uintptr_t>(M * L.N) * 2u;
+    bool xr = i > 0 && nrun < kRunMax;
+    for (int r = 0; r < nrun; ++r) xr = xr && !(xa < run_hi[r] && run_lo[r] < xb);
+    if (!xr) nrun = 0;
+    run_lo[nrun] = ya;
+    run_hi[nrun] = yb;
+    ++nrun;
+    if (run(i, s, xr) != cudaSuccess) return MPW_E_CUDA;
   }
   return MPW_OK;
 }

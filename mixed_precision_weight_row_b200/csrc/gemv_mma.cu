@@ -120,9 +120,6 @@ gemv_mma_kernel(const uint16_t* __restrict__ x, int M, const uint8_t* __restrict
   __shared__ float ss_red[kWarps][NS];
   __shared__ float cl_ss[8][NS];
 
-  // The next kernel in the stream may launch right away: it only reads its
-  // own weights until it passes griddepcontrol.wait.
-  asm volatile("griddepcontrol.launch_dependents;");
   cg::cluster_group cluster = cg::this_cluster();
   const int KC = static_cast<int>(cluster.num_blocks());
   const int cr = static_cast<int>(cluster.block_rank());
@@ -232,8 +229,10 @@ gemv_mma_kernel(const uint16_t* __restrict__ x, int M, const uint8_t* __restrict
     load_words_vec<B>(pb + sb, w1b);
   }
   // everything above reads only the weights; x may still be being written by
-  // the previous kernel in the stream
+  // the previous kernel in the stream.  The next kernel may launch once this
+  // wait has returned.
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (n_main > 0) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) load_x_vec(px[nt], x0[nt]);

@@ -26,10 +26,10 @@
 // resets the counter to zero for the next call.  No CTA ever waits for
 // another.
 //
-// Programmatic dependent launch: the next kernel in the stream may launch at
-// once; the producer issues the weight loads of the first stages before
-// griddepcontrol.wait and the x loads after it, and the thread that writes y
-// or the workspace waits first.  Every mbarrier wait is bounded (2 s); on
+// Programmatic dependent launch: the producer issues the weight loads of the
+// first stages before griddepcontrol.wait and the x loads after it, and lets
+// the next kernel in the stream launch once the wait has returned; the thread
+// that writes y or the workspace waits first.  Every mbarrier wait is bounded (2 s); on
 // time-out the kernel records an error in the device error word.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -159,7 +159,6 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   __shared__ float ss_red[2][kCW][NS];
   __shared__ __align__(16) uint4 zero_x[4];   // x fragment of lanes without a token
 
-  asm volatile("griddepcontrol.launch_dependents;");
   const int G = static_cast<int>(gridDim.x);
   const int b = static_cast<int>(blockIdx.x);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -204,7 +203,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       it.init(u0, u1, C);
       int pre = 0;
       for (; pre < S && it.valid(); ++pre, it.next()) issue_w(it, pre);
-      asm volatile("griddepcontrol.wait;" ::: "memory");
+      ptx::grid_dep_wait_then_release();
       StageIt ix;
       ix.init(u0, u1, C);
       for (int s = 0; s < pre; ++s, ix.next()) issue_x(ix, s);

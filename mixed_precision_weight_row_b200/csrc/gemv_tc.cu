@@ -29,7 +29,8 @@
 //     squares are gathered in the first CTA through distributed shared
 //     memory, which applies the row scale (and the rms scale) and writes y.
 // The weight loads of the first blocks are issued before
-// griddepcontrol.wait (programmatic dependent launch).  Every mbarrier wait
+// griddepcontrol.wait (programmatic dependent launch); the next kernel in
+// the stream may launch once that wait has returned.  Every mbarrier wait
 // is bounded; on time-out the kernel records an error in the device error
 // word and every role falls through to the final barriers.
 #include <cooperative_groups.h>
@@ -120,7 +121,6 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   auto empty_a = [&](int s) { return bar0 + 8u * (2 * SX + 2 * SW + SA + s); };
   const uint32_t acc_full = bar0 + 8u * (2 * SX + 2 * SW + 2 * SA);
 
-  asm volatile("griddepcontrol.launch_dependents;");
   cg::cluster_group cluster = cg::this_cluster();
   const int KC = static_cast<int>(cluster.num_blocks());
   const int cr = static_cast<int>(cluster.block_rank());
@@ -170,7 +170,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
   if (warp == 0) {
     // ---------------- x producer ----------------
     if (lane == 0) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");
+      ptx::grid_dep_wait_then_release();
       int issued = 0;
       for (int i = 0; i < nkb; ++i) {
         const int s = i % SX;

@@ -9,11 +9,15 @@
 // quantization tutorial, closing note).
 //
 // A CTA owns a 16-row tile of W (a cluster of 1..8 CTAs splits the tile's K
-// range).  The last warp is the producer: one lane walks the CTA's 128-code
-// chunks and, per chunk, issues one 2D TMA of the packed rows ({16*B bytes x
-// 16 rows}) and one of x ({128 values x M tokens}) into a ring of stages of
-// kCW*kCH chunks each (mbarrier completion; rows past N, bytes past the row
-// and values past K read as zeros).  Consumer warp w takes kCH consecutive
+// range).  The last warp is the producer: one lane fills a ring of stages of
+// kCW*kCH 128-code chunks each (mbarrier completion).  When K % 128 == 0 a
+// stage is two 3D TMAs: the packed rows viewed as [chunk][row][16*B bytes]
+// ({16*B x 16 rows x 8 chunks}) and x viewed as [chunk][token][128 values]
+// ({128 x M x 8 chunks}); rows past N and chunks past K read as zeros.  One
+// thread issuing many small copies is slow (tens of nanoseconds each), so
+// large boxes matter.  Other K take one 2D TMA per chunk and operand (bytes
+// past the row and values past K read as zeros).  Shared memory holds the
+// same [chunk][row] and [chunk][token] layout either way.  Consumer warp w takes kCH consecutive
 // chunks of each stage: per chunk, the 32-code group of lane tig for rows g
 // and g+8 (B words per row) and its x fragment for token g, both from shared
 // memory; it expands the codes to exact bf16 (expand.cuh; canonical or
@@ -22,12 +26,19 @@
 // memory and distributed shared memory into the cluster's first CTA, which
 // applies the row scale (and the rms scale with norm_input) and writes bf16.
 //
-// Programmatic dependent launch: every thread lets the next kernel launch at
-// once.  The producer issues the weight loads of the first stages before
-// griddepcontrol.wait and the x loads after it; the thread that writes y
-// waits too.  In a chain of linears the next layer's weights stream in while
-// the previous kernel drains.  Every mbarrier wait is bounded (2 s), after
-// which the kernel records an error in the device error word and winds down.
+// Programmatic dependent launch: the producer issues the weight loads of the
+// first stages before griddepcontrol.wait and the x loads after it, then
+// lets the next kernel in the stream launch; the thread that writes y waits
+// too.  In a chain of linears the next layer's weights stream in while this
+// kernel computes.  Because a CTA lets the next kernel launch only after its
+// own wait has returned, every launch before that wait's kernel is complete
+// when the next kernel starts.  With kXReady the caller states that x was
+// written before the launch that precedes the current run of such calls;
+// the kernel then lets the next one launch at once and loads x with the
+// weights, without waiting, so that consecutive calls overlap in full; only
+// the write of y waits for the predecessor.  Every mbarrier wait is bounded
+// (2 s), after which the kernel records an error in the device error word
+// and winds down.
 #include <cooperative_groups.h>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -55,6 +66,8 @@ constexpr int kThreads = (kCW + 1) * 32;
 constexpr int kChunk = 128;             // codes per chunk and row
 constexpr int kNormMaxM = 8;
 constexpr int kMaxStages = 8;
+constexpr int kXReady = 1;              // flags: x is not written by the preceding launch
+constexpr int kStageBoxes = 2;          // flags: one 3D TMA per stage and operand
 
 // Bytes of one stage: kSC weight chunks (16 rows x 16*B bytes) followed by
 // kSC x chunks (M tokens x 128 bf16).
@@ -62,10 +75,11 @@ __host__ __device__ constexpr uint32_t stage_bytes(int B, int M) {
   return static_cast<uint32_t>(kSC) * 256u * static_cast<uint32_t>(B + M);
 }
 
-// Ring depth.  With at most two CTAs per SM, a CTA whose whole K slice fits
-// in kWholeSlice bytes puts every stage of it in flight at once (latency
-// decides); otherwise two stages keep shared memory per CTA small and the
-// number of resident CTAs per SM high (occupancy decides).
+// Ring depth.  When the grid fits on the SMs in one wave, a CTA whose whole
+// K slice fits in kWholeSlice bytes puts every stage of it in flight at once
+// (latency decides); otherwise two stages keep shared memory per CTA small
+// and the number of resident CTAs per SM high (occupancy decides: CTAs of
+// the next launches become resident early and stream their weights).
 // MPW_GEMV_RING_KB replaces the rule by a fixed budget (tuning aid).
 constexpr uint32_t kWholeSlice = 64u * 1024u;
 
@@ -117,7 +131,7 @@ template <int B, int NT, bool NORM, bool PAIRED>
 __global__ void __launch_bounds__(kThreads, min_ctas<B, NT>())
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                 int M, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
-                int32_t* err) {
+                int flags, int32_t* err) {
   constexpr int P = Exp<B>::parts;
   constexpr int NS = NORM ? kNormMaxM : 1;
   constexpr uint32_t kWChunk = 256u * B;        // 16 rows x 16*B bytes
@@ -132,7 +146,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
   __shared__ float cl_ss[8][NS];
   __shared__ __align__(16) uint4 zero_x[4];   // x fragment of lanes without a token
 
-  asm volatile("griddepcontrol.launch_dependents;");
+  if (flags & kXReady) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cg::cluster_group cluster = cg::this_cluster();
   const int KC = static_cast<int>(cluster.num_blocks());
   const int cr = static_cast<int>(cluster.block_rank());
@@ -165,24 +179,44 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
     if (lane == 0) {
       ptx::prefetch_tmap(&tmap_w);
       ptx::prefetch_tmap(&tmap_x);
+      const bool boxes = (flags & kStageBoxes) != 0;
       auto nvalid = [&](int s) { return min(kSC, ce - (cb + kSC * s)); };
       auto issue_w = [&](int s, int slot) {
         const int c0 = cb + kSC * s, nv = nvalid(s);
+        if (boxes) {
+          // a box lands whole (zeros past the tensor); chunks past this
+          // CTA's range are loaded and not read
+          ptx::mbar_arrive_expect_tx(full(slot), st_bytes);
+          ptx::tma_load_3d(base + slot * st_bytes, &tmap_w, full(slot), 0, r0, c0);
+          return;
+        }
         ptx::mbar_arrive_expect_tx(full(slot), nv * (kWChunk + x_chunk));
         for (int j = 0; j < nv; ++j)
           ptx::tma_load_2d(base + slot * st_bytes + j * kWChunk, &tmap_w, full(slot), (c0 + j) * 16 * B, r0);
       };
       auto issue_x = [&](int s, int slot) {
         const int c0 = cb + kSC * s, nv = nvalid(s);
+        if (boxes) {
+          ptx::tma_load_3d(base + slot * st_bytes + w_part, &tmap_x, full(slot), 0, 0, c0);
+          return;
+        }
         for (int j = 0; j < nv; ++j)
           ptx::tma_load_2d(base + slot * st_bytes + w_part + j * x_chunk, &tmap_x, full(slot),
                            (c0 + j) * kChunk, 0);
       };
       const int pre = min(S, n_stages);
       // weights do not depend on the previous kernel in the stream; x does
-      for (int s = 0; s < pre; ++s) issue_w(s, s);
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      for (int s = 0; s < pre; ++s) issue_x(s, s);
+      // unless the caller says otherwise
+      if (flags & kXReady) {
+        for (int s = 0; s < pre; ++s) {
+          issue_w(s, s);
+          issue_x(s, s);
+        }
+      } else {
+        for (int s = 0; s < pre; ++s) issue_w(s, s);
+        ptx::grid_dep_wait_then_release();
+        for (int s = 0; s < pre; ++s) issue_x(s, s);
+      }
       int issued = pre;
       int slot = 0;
       uint32_t phase = 0;   // phase of empty(slot) that frees it for stage s
@@ -434,37 +468,61 @@ int cluster_size(int tiles, int chunks, int num_sms) {
 
 template <int B, int NT, bool NORM, bool PAIRED>
 cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
-                    uint16_t* y, bool pdl, int32_t* err, cudaStream_t stream) {
+                    uint16_t* y, bool pdl, int flags, int32_t* err, cudaStream_t stream) {
   auto encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
   const int64_t rb = 16 * ((static_cast<int64_t>(K) * B + 127) / 128);
+  const int chunks = (K + kChunk - 1) / kChunk;
   CUtensorMap tmap_w, tmap_x;
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(N)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(rb)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(16 * B), 16};
-    const cuuint32_t estr[2] = {1, 1};
-    if (encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return cudaErrorInvalidValue;
+  // Whole-stage boxes need every chunk of a row inside the row (K % 128 ==
+  // 0: rb == chunks * 16 * B), so that no in-bounds coordinate of the 3D
+  // views addresses past the buffers.
+  bool boxes = K % kChunk == 0;
+  if (boxes) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(16 * B), static_cast<cuuint64_t>(N),
+                                static_cast<cuuint64_t>(chunks)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(16 * B)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(16 * B), 16, static_cast<cuuint32_t>(kSC)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    boxes = encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(packed), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   }
-  {
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(M)};
+  if (boxes) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kChunk), static_cast<cuuint64_t>(M),
+                                static_cast<cuuint64_t>(chunks)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(kChunk) * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(M),
+                               static_cast<cuuint32_t>(kSC)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    boxes = encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
+  if (boxes) {
+    flags |= kStageBoxes;
+  } else {
+    // one 2D TMA per chunk: {16*B bytes x 16 rows} of W, {128 values x M} of x
+    const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(N)};
+    const cuuint64_t wstrides[1] = {static_cast<cuuint64_t>(rb)};
+    const cuuint32_t wbox[2] = {static_cast<cuuint32_t>(16 * B), 16};
+    const cuuint64_t xdims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t xstrides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t xbox[2] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(M)};
     const cuuint32_t estr[2] = {1, 1};
-    if (encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides, box,
+    if (encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), wdims, wstrides, wbox,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), xdims, xstrides, xbox,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
   auto kern = gemv_tma_kernel<B, NT, NORM, PAIRED>;
   const int tiles = (N + 15) / 16;
-  const int chunks = (K + kChunk - 1) / kChunk;
   const int kc = cluster_size(tiles, chunks, device_info().num_sms);
   const int per_cta = ((chunks + kc - 1) / kc + kSC - 1) / kSC;
-  const int S = ring_stages(B, M, per_cta, tiles * kc <= 2 * device_info().num_sms);
+  const int S = ring_stages(B, M, per_cta, tiles * kc <= device_info().num_sms);
   const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M);
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
@@ -487,34 +545,35 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
   }
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, tmap_w, tmap_x, M, scales, N, K, y, S, err);
+  return cudaLaunchKernelEx(&cfg, kern, tmap_w, tmap_x, M, scales, N, K, y, S, flags, err);
 }
 
 template <int B, bool PAIRED>
 cudaError_t tma_bits(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
-                     uint16_t* y, bool norm, bool pdl, int32_t* err, cudaStream_t stream) {
-  if (norm) return run_tma<B, 1, true, PAIRED>(x, M, packed, scales, N, K, y, pdl, err, stream);  // M <= 8
-  if (M <= 8) return run_tma<B, 1, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, err, stream);
-  if (M <= 16) return run_tma<B, 2, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, err, stream);
-  return run_tma<B, 4, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, err, stream);
+                     uint16_t* y, bool norm, bool pdl, int flags, int32_t* err, cudaStream_t stream) {
+  if (norm) return run_tma<B, 1, true, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);  // M <= 8
+  if (M <= 8) return run_tma<B, 1, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  if (M <= 16) return run_tma<B, 2, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  return run_tma<B, 4, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
 }
 
 template <bool PAIRED>
 cudaError_t tma_layout(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int bits, int N,
-                       int K, uint16_t* y, bool norm, bool pdl, int32_t* err, cudaStream_t stream) {
+                       int K, uint16_t* y, bool norm, bool pdl, int flags, int32_t* err,
+                       cudaStream_t stream) {
   switch (bits) {
-    case 4: return tma_bits<4, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 5: return tma_bits<5, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 6: return tma_bits<6, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 7: return tma_bits<7, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 8: return tma_bits<8, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 9: return tma_bits<9, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 10: return tma_bits<10, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 11: return tma_bits<11, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 12: return tma_bits<12, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 13: return tma_bits<13, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 14: return tma_bits<14, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
-    case 15: return tma_bits<15, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, err, stream);
+    case 4: return tma_bits<4, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 5: return tma_bits<5, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 6: return tma_bits<6, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 7: return tma_bits<7, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 8: return tma_bits<8, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 9: return tma_bits<9, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 10: return tma_bits<10, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 11: return tma_bits<11, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 12: return tma_bits<12, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 13: return tma_bits<13, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 14: return tma_bits<14, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
+    case 15: return tma_bits<15, PAIRED>(x, M, packed, scales, N, K, y, norm, pdl, flags, err, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -530,12 +589,13 @@ bool gemv_tma_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, bool
 
 cudaError_t launch_gemv_tma(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
                             int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, bool pdl,
-                            cudaStream_t stream) {
+                            bool x_ready, cudaStream_t stream) {
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   int32_t* err = device_error_word();
+  const int flags = x_ready ? kXReady : 0;
   if (layout == kLayoutPaired)
-    return tma_layout<true>(x, m, packed, scales, bits, n, k, y, norm, pdl, err, stream);
-  return tma_layout<false>(x, m, packed, scales, bits, n, k, y, norm, pdl, err, stream);
+    return tma_layout<true>(x, m, packed, scales, bits, n, k, y, norm, pdl, flags, err, stream);
+  return tma_layout<false>(x, m, packed, scales, bits, n, k, y, norm, pdl, flags, err, stream);
 }
 
 }  // namespace mpw

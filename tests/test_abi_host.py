@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
                  "mpw_qlinear_path", "mpw_recipe_run", "mpw_packed_row_bytes",
                  "mpw_status_str", "mpw_version", "mpw_device_error", "mpw_repack",
                  "mpw_qlinear_ex", "mpw_qlinear_ws", "mpw_qlinear_workspace_bytes",
-                 "mpw_recipe_run_ws", "mpw_recipe_workspace_bytes"):
+                 "mpw_recipe_run_ws", "mpw_recipe_workspace_bytes", "mpw_qlinear_flags"):
         assert want in names
 
 
@@ -127,6 +127,28 @@ def test_qlinear_ex_validation():
     assert L.mpw_qlinear_ex(A16 + 2, A16B, A16, 5, 1, 1, 4, 64, A16, 0, 0) == mpw.MPW_E_MISALIGNED
     assert L.mpw_qlinear_ex(A16, A16B, A16, 5, 1, 1, 4, 64, A16, 3, 0) == mpw.MPW_E_INVALID_ARG
     assert L.mpw_qlinear_ex(A16, A16B, A16, 2, 1, 1, 4, 64, A16, 0, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+
+
+def test_qlinear_flags_validation():
+    L = mpw.lib
+    # unknown flag bits are an argument error; the usual checks still apply
+    assert L.mpw_qlinear_flags(A16, A16B, A16, 5, 1, 1, 4, 64, A16, 0, 2, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_flags(A16, A16B, A16, 5, 1, 1, 4, 64, A16, 0, 0x80000000, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_flags(A16, A16B, A16, 3, 1, 1, 4, 64, A16, 0, mpw.X_READY, 0) == \
+        mpw.MPW_E_UNSUPPORTED_BITS
+    assert L.mpw_qlinear_flags(A16 + 2, A16B, A16, 5, 1, 1, 4, 64, A16, 0, mpw.X_READY, 0) == \
+        mpw.MPW_E_MISALIGNED
+    assert L.mpw_qlinear_flags(A16, A16B, A16, 5, 1, 1, 4, 48, A16, 0, mpw.X_READY, 0) == mpw.MPW_E_INVALID_ARG
+
+
+def test_binding_rejects_x_ready_with_workspace():
+    import torch
+
+    x = torch.zeros((1, 64), dtype=torch.bfloat16)
+    p = torch.zeros((4, mpw.packed_row_bytes(64, 5)), dtype=torch.uint8)
+    s = torch.ones((4,), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        mpw.qlinear(x, p, s, 5, x_ready=True, use_workspace=True)
 
 
 def test_qlinear_ws_validation():
