@@ -510,6 +510,8 @@ def decode_config(args, pool):
             "pool_matrices": pool, "l2": "inputs larger than L2: rotating pool of distinct packed "
                                          "matrices totalling > 4x L2 per step",
             "parallelism": f"replicas x{args.gpus}",
+            "launches": "one qlinear call per matrix, back to back on one stream in a CUDA graph, each "
+                        "flagged x_ready (no launch writes x); dependent_chain times them unflagged",
             "layout": (f"{args.layout}" + (": paired-halves re-ordering of the canonical bits, same bytes, "
                                            "repacked once outside the timed region"
                                            if args.layout == "paired" else ""))}

@@ -141,12 +141,25 @@ constexpr int min_ctas() {
   return NT == 1 ? (B <= 7 ? 4 : 3) : (NT == 2 ? 2 : 1);
 }
 
+// Parts (MMAs per k step) of a code: paired rows take the combined scheme of
+// the prefill GEMM (one part up to b = 9, lo7 + 128 * hi above), canonical
+// rows the decode schemes of expand.cuh.
+template <int B, bool PAIRED>
+constexpr int dec_parts() {
+  return PAIRED ? GemmParts<B>::parts : Exp<B>::parts;
+}
+
+template <int B, int NT, bool PAIRED>
+constexpr int min_ctas_for() {
+  return dec_parts<B, PAIRED>() == 1 && NT == 1 ? 4 : min_ctas<B, NT>();
+}
+
 template <int B, int NT, bool NORM, bool PAIRED>
-__global__ void __launch_bounds__(kThreads, min_ctas<B, NT>())
+__global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, PAIRED>())
 gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x, int M,
                const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S, int64_t U,
                int kmax, float* __restrict__ ws_part, int* __restrict__ ws_cnt, int32_t* err) {
-  constexpr int P = Exp<B>::parts;
+  constexpr int P = dec_parts<B, PAIRED>();
   constexpr int NS = NORM ? kNormMaxM : 1;
   constexpr int SLOT = slot_floats<NT>();
   constexpr uint32_t kWChunk = 256u * B;        // 16 rows x 16*B bytes
@@ -272,8 +285,8 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     }
     uint32_t va[P][16], vb[P][16];
     if constexpr (PAIRED) {
-      expand_paired<B>(wa, va);
-      expand_paired<B>(wb, vb);
+      gemm_expand_group<B, true>(wa, va);
+      gemm_expand_group<B, true>(wb, vb);
     } else {
       expand_group<B>(wa, va);
       expand_group<B>(wb, vb);
