@@ -234,21 +234,23 @@ def decode_setup(mpw, W_gpu, b, l2_bytes, layout="canonical"):
 
 
 def measure_decode(mpw, pool, b, M, K, N, steps, warmup, world=1, x=None, layout="canonical", x_ready=True):
-    """Back-to-back launches over the pool's distinct matrices with one x.
-    No launch writes x, which each call states (x_ready) unless asked not to,
-    so that a launch's product may overlap its predecessor; x_ready=False
-    times the same launches as a dependent chain."""
+    """Back-to-back launches over the pool's distinct matrices with one x,
+    each writing its own output.  No launch writes x or another launch's y,
+    which each call states (x_ready, y_unshared) unless asked not to, so that
+    a launch overlaps its predecessors; x_ready=False times the same launches
+    as a dependent chain."""
     import torch
 
     import workloads as wl
 
     if x is None:
         x = wl.gen_x(M, K, wl.DECODE["x_seed"]).cuda()
-    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ys = torch.empty((pool.P, M, N), dtype=torch.bfloat16, device="cuda")
 
     def step():
         for i in range(pool.P):
-            mpw.qlinear(x, pool.packed[i], pool.scales[i], b, y=y, layout=layout, x_ready=x_ready)
+            mpw.qlinear(x, pool.packed[i], pool.scales[i], b, y=ys[i], layout=layout, x_ready=x_ready,
+                        y_unshared=x_ready)
 
     g = graph_of(step)
     ms = time_graph(g, steps, warmup, world)
@@ -511,7 +513,8 @@ def decode_config(args, pool):
                                          "matrices totalling > 4x L2 per step",
             "parallelism": f"replicas x{args.gpus}",
             "launches": "one qlinear call per matrix, back to back on one stream in a CUDA graph, each "
-                        "flagged x_ready (no launch writes x); dependent_chain times them unflagged",
+                        "into its own output and flagged x_ready + y_unshared (no launch writes x or "
+                        "another's y); dependent_chain times them unflagged",
             "layout": (f"{args.layout}" + (": paired-halves re-ordering of the canonical bits, same bytes, "
                                            "repacked once outside the timed region"
                                            if args.layout == "paired" else ""))}
@@ -564,12 +567,14 @@ def main(argv=None):
     lay = args.layout
     pool = decode_setup(mpw, W, HEADLINE_BITS, l2, lay)
     x1 = wl.gen_x(1, K, c["x_seed"]).cuda()
-    y1 = torch.empty((1, N), dtype=torch.bfloat16, device="cuda")
+    y1 = torch.empty((pool.P, 1, N), dtype=torch.bfloat16, device="cuda")
 
     def step():
-        # distinct matrices applied to one x: no launch writes x (x_ready)
+        # distinct matrices applied to one x, each into its own output: no
+        # launch writes x or another launch's y (x_ready, y_unshared)
         for i in range(pool.P):
-            mpw.qlinear(x1, pool.packed[i], pool.scales[i], HEADLINE_BITS, y=y1, layout=lay, x_ready=True)
+            mpw.qlinear(x1, pool.packed[i], pool.scales[i], HEADLINE_BITS, y=y1[i], layout=lay, x_ready=True,
+                        y_unshared=True)
 
     g = graph_of(step)
     with ClockSampler(uuid) as cs:

@@ -202,8 +202,9 @@ MPW_API mpw_status mpw_qlinear_ws(const uint16_t* x, const uint8_t* packed, cons
                                   mpw_stream_t stream);
 
 /*
- * mpw_qlinear_flags -- mpw_qlinear_ex with flags (0 or MPW_QLINEAR_X_READY;
- * other bits are MPW_E_INVALID_ARG).
+ * mpw_qlinear_flags -- mpw_qlinear_ex with flags (0, MPW_QLINEAR_X_READY or
+ * MPW_QLINEAR_X_READY | MPW_QLINEAR_Y_UNSHARED; other bits are
+ * MPW_E_INVALID_ARG).
  *   MPW_QLINEAR_X_READY: the caller states that x was written before the
  *   launch that precedes the current run of flagged calls on `stream` (the
  *   consecutive calls made with this flag, this one included): neither a
@@ -222,6 +223,17 @@ MPW_API mpw_status mpw_qlinear_ws(const uint16_t* x, const uint8_t* packed, cons
  *   x), not an error code.  Results are those of mpw_qlinear_ex.
  */
 #define MPW_QLINEAR_X_READY 1u
+/*
+ *   MPW_QLINEAR_Y_UNSHARED (only with MPW_QLINEAR_X_READY, else
+ *   MPW_E_INVALID_ARG): the caller also states that no other call of the run
+ *   and not the launch just before it reads or writes y (q, k and v writing
+ *   three different buffers; distinct outputs for a set of matrices).  The
+ *   kernel then writes y without waiting for its predecessor; one of its
+ *   blocks still waits, so kernels complete in launch order and an unflagged
+ *   call after the run sees every output of it.  A false statement is a data
+ *   race, not an error code.
+ */
+#define MPW_QLINEAR_Y_UNSHARED 2u
 MPW_API mpw_status mpw_qlinear_flags(const uint16_t* x, const uint8_t* packed, const float* scales,
                                      int bits, int layout, int64_t M, int64_t N, int64_t K,
                                      uint16_t* y, int path, unsigned flags, mpw_stream_t stream);
@@ -260,8 +272,9 @@ typedef struct mpw_linear {
  * graph).  A linear whose input bytes were written neither by the linear
  * before the current run of such linears nor by one inside it (k and v after
  * q; up after gate) is launched with MPW_QLINEAR_X_READY, so that it runs
- * alongside its predecessors; the first linear never is.  Outputs land in
- * order.  slots[i] are device bf16 buffers; each must hold M * (largest N or
+ * alongside its predecessors, and also with MPW_QLINEAR_Y_UNSHARED when its
+ * output bytes are neither read nor written by that run and linear; the
+ * first linear is never flagged.  slots[i] are device bf16 buffers; each must hold M * (largest N or
  * K that touches it) elements.  M must be in 1..32 (the decode pass).
  * A linear whose in_slot equals its out_slot is rejected.
  */

@@ -39,6 +39,8 @@ LAYOUTS = {"canonical": 0, "paired": 1}
 # mpw_qlinear_flags: x was written before the launch preceding the run of
 # flagged calls
 X_READY = 1
+# with X_READY: no other call of the run, nor the launch before it, touches y
+Y_UNSHARED = 2
 
 
 class MPWError(RuntimeError):
@@ -256,7 +258,7 @@ def repack(packed, K: int, bits: int, layout_in: str = "canonical", layout_out: 
 
 
 def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: str = "canonical",
-            stream=None, use_workspace: bool = False, x_ready: bool = False):
+            stream=None, use_workspace: bool = False, x_ready: bool = False, y_unshared: bool = False):
     """y = x @ (q * s)^T with x bf16 [M, K]; returns y bf16 [M, N].
 
     With ``use_workspace`` the decode path (M <= 32) gets this stream's
@@ -264,11 +266,15 @@ def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: st
     on every measured shape) the per-tile kernel.  ``x_ready`` states that x
     was written before the launch that precedes the current run of x_ready
     calls on the stream (MPW_QLINEAR_X_READY in mpw.h); it cannot be combined
-    with a workspace."""
+    with a workspace.  ``y_unshared`` (only with ``x_ready``) states that no
+    other call of that run, nor the launch before it, reads or writes y
+    (MPW_QLINEAR_Y_UNSHARED)."""
     import torch
 
     if x_ready and use_workspace:
         raise ValueError("x_ready cannot be combined with use_workspace")
+    if y_unshared and not x_ready:
+        raise ValueError("y_unshared needs x_ready")
     _need(x, torch.bfloat16, "x", 2)
     _need(packed, torch.uint8, "packed", 2)
     _need(scales, torch.float32, "scales", 1)
@@ -283,7 +289,8 @@ def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: st
     _need(y, torch.bfloat16, "y")
     if x_ready:
         _check(lib.mpw_qlinear_flags(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits),
-                                     LAYOUTS[layout], M, N, K, y.data_ptr(), PATHS[path], X_READY,
+                                     LAYOUTS[layout], M, N, K, y.data_ptr(), PATHS[path],
+                                     X_READY | (Y_UNSHARED if y_unshared else 0),
                                      _stream(stream)), "mpw_qlinear_flags")
         return y
     ws, ws_bytes = None, 0

@@ -47,11 +47,15 @@ const DeviceInfo& device_info() {
   if (d.device != dev) {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (d.device != dev) {
-      int sms = 0, smem = 0;
+      int sms = 0, smem = 0, per_sm = 0, reserved = 0;
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
       cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
       d.num_sms = sms > 0 ? sms : 1;
       d.max_smem_optin = smem;
+      d.smem_per_sm = per_sm;
+      d.smem_reserved = reserved;
       d.device = dev;
     }
   }
@@ -174,7 +178,8 @@ mpw_status qlinear_impl(const uint16_t* x, const uint8_t* packed, const float* s
                         int64_t M, int64_t N, int64_t K, uint16_t* y, int path, void* ws, size_t ws_bytes,
                         unsigned flags, mpw_stream_t stream) {
   if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
-  if ((flags & ~static_cast<unsigned>(MPW_QLINEAR_X_READY)) != 0) return MPW_E_INVALID_ARG;
+  if ((flags & ~static_cast<unsigned>(MPW_QLINEAR_X_READY | MPW_QLINEAR_Y_UNSHARED)) != 0) return MPW_E_INVALID_ARG;
+  if ((flags & MPW_QLINEAR_Y_UNSHARED) && !(flags & MPW_QLINEAR_X_READY)) return MPW_E_INVALID_ARG;
   if (x == nullptr || packed == nullptr || scales == nullptr || y == nullptr || M < 1 || N < 1 ||
       K < 1)
     return MPW_E_INVALID_ARG;
@@ -192,8 +197,9 @@ mpw_status qlinear_impl(const uint16_t* x, const uint8_t* packed, const float* s
   }
   if (path == MPW_PATH_GEMM) return MPW_E_INVALID_ARG;  // shape the GEMM does not take
   if (ws != nullptr && ws_bytes < gemv_workspace_bytes(x, bits, layout, M, N, K, false)) return MPW_E_INVALID_ARG;
-  return from_cuda(launch_gemv(x, packed, scales, bits, layout, M, N, K, y, false, ws, ws_bytes, s,
-                               (flags & MPW_QLINEAR_X_READY) != 0));
+  static_assert(MPW_QLINEAR_X_READY == kQlinearXReady && MPW_QLINEAR_Y_UNSHARED == kQlinearYFree,
+                "flag values");
+  return from_cuda(launch_gemv(x, packed, scales, bits, layout, M, N, K, y, false, ws, ws_bytes, s, flags));
 }
 
 }  // namespace
@@ -284,32 +290,42 @@ mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count, uint16_t* 
     if (workspace_bytes < recipe_ws_bytes(layers, count, M)) return MPW_E_INVALID_ARG;
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  auto run = [&](int64_t i, cudaStream_t st, bool x_ready) {
+  auto run = [&](int64_t i, cudaStream_t st, unsigned qflags) {
     const mpw_linear& L = layers[i];
     return launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, L.layout, M, L.N, L.K, slots[L.out_slot],
-                       L.norm_input != 0, workspace, workspace_bytes, st, x_ready);
+                       L.norm_input != 0, workspace, workspace_bytes, st, qflags);
   };
   // A linear whose input was written neither by the linear before the
   // current run of x-ready linears nor by one inside it joins the run
-  // (MPW_QLINEAR_X_READY): k and v after q, up after gate.  Inputs and
-  // outputs are compared as byte ranges, so slots that alias are safe.  The
-  // first linear follows whatever the caller launched before: never.
+  // (MPW_QLINEAR_X_READY): k and v after q, up after gate; when its output is
+  // also neither read nor written by the run and that linear, it writes it
+  // without waiting (MPW_QLINEAR_Y_UNSHARED).  Inputs and outputs are
+  // compared as byte ranges, so slots that alias are safe.  The first linear
+  // follows whatever the caller launched before: never.
   constexpr int kRunMax = 8;
-  uintptr_t run_lo[kRunMax], run_hi[kRunMax];  // outputs of the run and of the linear before it
+  // inputs and outputs of the run and of the linear before it
+  uintptr_t in_lo[kRunMax], in_hi[kRunMax], out_lo[kRunMax], out_hi[kRunMax];
   int nrun = 0;
+  auto overlaps = [&](const uintptr_t* lo, const uintptr_t* hi, uintptr_t a, uintptr_t b) {
+    for (int r = 0; r < nrun; ++r)
+      if (a < hi[r] && lo[r] < b) return true;
+    return false;
+  };
   for (int64_t i = 0; i < count; ++i) {
     const mpw_linear& L = layers[i];
     const uintptr_t xa = reinterpret_cast<uintptr_t>(slots[L.in_slot]);
     const uintptr_t xb = xa + static_cast<uintptr_t>(M * L.K) * 2u;
     const uintptr_t ya = reinterpret_cast<uintptr_t>(slots[L.out_slot]);
     const uintptr_t yb = ya + static_cast<uintptr_t>(M * L.N) * 2u;
-    bool xr = i > 0 && nrun < kRunMax;
-    for (int r = 0; r < nrun; ++r) xr = xr && !(xa < run_hi[r] && run_lo[r] < xb);
+    const bool xr = i > 0 && nrun < kRunMax && !overlaps(out_lo, out_hi, xa, xb);
+    const bool yf = xr && !overlaps(out_lo, out_hi, ya, yb) && !overlaps(in_lo, in_hi, ya, yb);
     if (!xr) nrun = 0;
-    run_lo[nrun] = ya;
-    run_hi[nrun] = yb;
+    in_lo[nrun] = xa;
+    in_hi[nrun] = xb;
+    out_lo[nrun] = ya;
+    out_hi[nrun] = yb;
     ++nrun;
-    if (run(i, s, xr) != cudaSuccess) return MPW_E_CUDA;
+    if (run(i, s, (xr ? kQlinearXReady : 0u) | (yf ? kQlinearYFree : 0u)) != cudaSuccess) return MPW_E_CUDA;
   }
   return MPW_OK;
 }

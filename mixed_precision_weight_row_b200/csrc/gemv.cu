@@ -457,7 +457,7 @@ size_t gemv_workspace_bytes(const uint16_t* x_or_null, int bits, int layout, int
 
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
                         int layout, int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm_input,
-                        void* ws, size_t ws_bytes, cudaStream_t stream, bool x_ready) {
+                        void* ws, size_t ws_bytes, cudaStream_t stream, unsigned qflags) {
   // Tensor-core decode kernels in passes of up to 32 tokens (8 with
   // norm_input): the stream-K kernel when a workspace is given, else the
   // per-tile TMA kernel.  MPW_GEMV_KERNEL=mma selects the register-streaming
@@ -502,7 +502,7 @@ cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* s
       if (e != cudaSuccess) return e;
       if (!used)
         e = tma ? launch_gemv_tma(x + m0 * K, packed, scales, bits, layout, mt, N, K, y + m0 * N, norm_input,
-                                  /*pdl=*/true, x_ready, stream)
+                                  /*pdl=*/true, qflags, stream)
                 : launch_gemv_mma(x + m0 * K, packed, scales, bits, mt, N, K, y + m0 * N, norm_input,
                                   /*pdl=*/true, stream);
       if (e != cudaSuccess) return e;

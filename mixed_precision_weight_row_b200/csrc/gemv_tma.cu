@@ -36,7 +36,10 @@
 // written before the launch that precedes the current run of such calls;
 // the kernel then lets the next one launch at once and loads x with the
 // weights, without waiting, so that consecutive calls overlap in full; only
-// the write of y waits for the predecessor.  Every mbarrier wait is bounded
+// the write of y waits for the predecessor.  With kYFree as well (no call of
+// the run, nor the launch before it, reads or writes y) only the first CTA
+// waits before writing, which keeps completions in launch order, and every
+// other CTA writes y and exits at once.  Every mbarrier wait is bounded
 // (2 s), after which the kernel records an error in the device error word
 // and winds down.
 #include <cooperative_groups.h>
@@ -68,6 +71,7 @@ constexpr int kNormMaxM = 8;
 constexpr int kMaxStages = 8;
 constexpr int kXReady = 1;              // flags: x is not written by the preceding launch
 constexpr int kStageBoxes = 2;          // flags: one 3D TMA per stage and operand
+constexpr int kYFree = 4;               // flags: no call of the run touches y
 
 // Bytes of one stage: kSC weight chunks (16 rows x 16*B bytes) followed by
 // kSC x chunks (M tokens x 128 bf16).
@@ -77,13 +81,15 @@ __host__ __device__ constexpr uint32_t stage_bytes(int B, int M) {
 
 // Ring depth.  When the grid fits on the SMs in one wave, a CTA whose whole
 // K slice fits in kWholeSlice bytes puts every stage of it in flight at once
-// (latency decides); otherwise two stages keep shared memory per CTA small
-// and the number of resident CTAs per SM high (occupancy decides: CTAs of
-// the next launches become resident early and stream their weights).
+// (latency decides).  Otherwise the register-limited number of resident CTAs
+// per SM decides (CTAs of the next launches become resident early and stream
+// their weights): the ring takes as many stages (at least two) as keep that
+// many CTAs in shared memory, and no more than the CTA's slice needs.
+// `fixed` is the shared memory a CTA needs besides its ring.
 // MPW_GEMV_RING_KB replaces the rule by a fixed budget (tuning aid).
 constexpr uint32_t kWholeSlice = 64u * 1024u;
 
-int ring_stages(int B, int M, int stages_per_cta, bool few_ctas) {
+int ring_stages(int B, int M, int stages_per_cta, bool few_ctas, int ctas_by_regs, uint32_t fixed) {
   static const uint32_t budget = [] {
     const char* e = getenv("MPW_GEMV_RING_KB");
     const int v = e ? atoi(e) : 0;
@@ -91,10 +97,16 @@ int ring_stages(int B, int M, int stages_per_cta, bool few_ctas) {
   }();
   const uint32_t st = stage_bytes(B, M);
   int s;
-  if (budget != 0)
+  if (budget != 0) {
     s = static_cast<int>(budget / st);
-  else
-    s = few_ctas && static_cast<uint32_t>(stages_per_cta) * st <= kWholeSlice ? stages_per_cta : 2;
+  } else if (few_ctas && static_cast<uint32_t>(stages_per_cta) * st <= kWholeSlice) {
+    s = stages_per_cta;
+  } else {
+    const DeviceInfo& d = device_info();
+    const int per_cta = ctas_by_regs > 0 ? d.smem_per_sm / ctas_by_regs - d.smem_reserved : 0;
+    s = per_cta > static_cast<int>(fixed) ? static_cast<int>((per_cta - fixed) / st) : 2;
+    if (s > stages_per_cta) s = stages_per_cta;
+  }
   return s < 2 ? 2 : (s > kMaxStages ? kMaxStages : s);
 }
 
@@ -135,13 +147,17 @@ constexpr int dec_parts() {
   return PAIRED ? GemmParts<B>::parts : Exp<B>::parts;
 }
 
-template <int B, int NT, bool PAIRED>
+// Paired rows with one part and one token tile fit in 64 registers (56 for
+// b <= 5): six or
+// seven CTAs per SM; the rms-scaled variant keeps eight sums of squares more
+// and stays at four.
+template <int B, int NT, bool NORM, bool PAIRED>
 constexpr int min_ctas_for() {
-  return dec_parts<B, PAIRED>() == 1 && NT == 1 ? 4 : min_ctas<B, NT>();
+  return PAIRED && dec_parts<B, PAIRED>() == 1 && NT == 1 ? (NORM ? 4 : 6) : min_ctas<B, NT>();
 }
 
 template <int B, int NT, bool NORM, bool PAIRED>
-__global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, PAIRED>())
+__global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, NORM, PAIRED>())
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                 int M, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
                 int flags, int32_t* err) {
@@ -151,13 +167,15 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
   const uint32_t x_chunk = 256u * M;            // M tokens x 128 bf16
   const uint32_t w_part = kSC * kWChunk;
   const uint32_t st_bytes = stage_bytes(B, M);
+  // dynamic: the ring (S stages), then, in clusters, the partial sums of the
+  // cluster's CTAs
   extern __shared__ __align__(128) uint8_t tsmem[];
   __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
   __shared__ float red[kCW][NT][32][4];
-  __shared__ float cl_red[8][NT][32][4];
   __shared__ float ss_red[kCW][NS];
   __shared__ float cl_ss[8][NS];
   __shared__ __align__(16) uint4 zero_x[4];   // x fragment of lanes without a token
+  auto cl_red = reinterpret_cast<float (*)[NT][32][4]>(tsmem + static_cast<uint32_t>(S) * stage_bytes(B, M));
 
   if (flags & kXReady) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cg::cluster_group cluster = cg::this_cluster();
@@ -427,8 +445,10 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
       const int ra = r0 + g, rb = r0 + g + 8;
       const float sca = ra < N ? __ldg(scales + ra) : 0.0f;
       const float scb = rb < N ? __ldg(scales + rb) : 0.0f;
-      // y may be read by the previous kernel in the stream
-      asm volatile("griddepcontrol.wait;" ::: "memory");
+      // y may be read or written by the previous kernel in the stream; with
+      // kYFree it is not, and the first CTA's wait alone keeps this kernel
+      // from completing before its predecessor
+      if (!(flags & kYFree) || blockIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -535,8 +555,18 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
   const int tiles = (N + 15) / 16;
   const int kc = cluster_size(tiles, chunks, device_info().num_sms);
   const int per_cta = ((chunks + kc - 1) / kc + kSC - 1) / kSC;
-  const int S = ring_stages(B, M, per_cta, tiles * kc <= device_info().num_sms);
-  const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M);
+  // resident CTAs per SM that registers and static shared memory allow
+  static const int ctas_by_regs = [] {
+    int n = 0;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tma_kernel<B, NT, NORM, PAIRED>, kThreads, 0) ==
+                   cudaSuccess
+               ? n
+               : 0;
+  }();
+  const uint32_t cl_bytes = kc > 1 ? static_cast<uint32_t>(kc) * NT * 32 * 4 * sizeof(float) : 0u;
+  const uint32_t fixed = cl_bytes + static_cast<uint32_t>(sizeof(float)) * kCW * NT * 32 * 4 + 1024u;
+  const int S = ring_stages(B, M, per_cta, tiles * kc <= device_info().num_sms, ctas_by_regs, fixed);
+  const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M) + cl_bytes;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -602,10 +632,11 @@ bool gemv_tma_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, bool
 
 cudaError_t launch_gemv_tma(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
                             int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, bool pdl,
-                            bool x_ready, cudaStream_t stream) {
+                            unsigned qflags, cudaStream_t stream) {
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   int32_t* err = device_error_word();
-  const int flags = x_ready ? kXReady : 0;
+  const bool x_ready = (qflags & kQlinearXReady) != 0;
+  const int flags = (x_ready ? kXReady : 0) | (x_ready && (qflags & kQlinearYFree) ? kYFree : 0);
   if (layout == kLayoutPaired)
     return tma_layout<true>(x, m, packed, scales, bits, n, k, y, norm, pdl, flags, err, stream);
   return tma_layout<false>(x, m, packed, scales, bits, n, k, y, norm, pdl, flags, err, stream);

@@ -26,6 +26,8 @@ struct DeviceInfo {
   int device = -1;
   int num_sms = 0;
   int max_smem_optin = 0;  // bytes of dynamic shared memory a block may opt into
+  int smem_per_sm = 0;     // bytes of shared memory per SM
+  int smem_reserved = 0;   // bytes the system reserves per resident block
 };
 const DeviceInfo& device_info();
 
@@ -54,13 +56,17 @@ cudaError_t launch_repack(const uint8_t* in, int64_t N, int64_t K, int bits, uin
 // gemv.cu: decode linear y[M, N] for any M (tensor-core kernels in passes of
 // 32 tokens; CUDA-core kernels for canonical shapes they do not take).  The
 // paired layout needs a shape the TMA kernel takes (checked by the caller).
-// x_ready: x was written before the launch that precedes the current run of
-// x_ready calls on the stream (MPW_QLINEAR_X_READY); the per-tile kernel then
-// releases its successor at once and loads x without waiting.
+// qflags: kQlinearXReady = x was written before the launch that precedes the
+// current run of such calls on the stream (MPW_QLINEAR_X_READY): the per-tile
+// kernel then releases its successor at once and loads x without waiting;
+// kQlinearYFree (with it) = no call of the run, nor the launch before it,
+// reads or writes y (MPW_QLINEAR_Y_UNSHARED): y is written without waiting.
+constexpr unsigned kQlinearXReady = 1u;
+constexpr unsigned kQlinearYFree = 2u;
 cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* scales,
                         int bits, int layout, int64_t M, int64_t N, int64_t K, uint16_t* y,
                         bool norm_input, void* ws, size_t ws_bytes, cudaStream_t stream,
-                        bool x_ready = false);
+                        unsigned qflags = 0u);
 // Workspace bytes launch_gemv uses for these arguments (0 if none).
 size_t gemv_workspace_bytes(const uint16_t* x_or_null, int bits, int layout, int64_t M, int64_t N,
                             int64_t K, bool norm_input);
@@ -79,11 +85,11 @@ cudaError_t launch_gemv_mma(const uint16_t* x, const uint8_t* packed, const floa
 
 // gemv_tma.cu: decode linear with the packed stream and x staged by TMA in a
 // shared-memory ring (the default decode kernel for M <= 32; needs K % 8 == 0
-// and a 16-byte aligned x).  x_ready as for launch_gemv.
+// and a 16-byte aligned x).  qflags as for launch_gemv.
 bool gemv_tma_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, bool norm);
 cudaError_t launch_gemv_tma(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
                             int layout, int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm,
-                            bool pdl, bool x_ready, cudaStream_t stream);
+                            bool pdl, unsigned qflags, cudaStream_t stream);
 
 // gemv_sk.cu: decode linear with the (tile, chunk) units split evenly over
 // a persistent grid; split tiles are combined in a caller workspace (zeroed

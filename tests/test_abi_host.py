@@ -139,6 +139,12 @@ def test_qlinear_flags_validation():
     assert L.mpw_qlinear_flags(A16 + 2, A16B, A16, 5, 1, 1, 4, 64, A16, 0, mpw.X_READY, 0) == \
         mpw.MPW_E_MISALIGNED
     assert L.mpw_qlinear_flags(A16, A16B, A16, 5, 1, 1, 4, 48, A16, 0, mpw.X_READY, 0) == mpw.MPW_E_INVALID_ARG
+    # y_unshared needs x_ready; bit 2 is not a flag
+    assert L.mpw_qlinear_flags(A16, A16B, A16, 5, 1, 1, 4, 64, A16, 0, mpw.Y_UNSHARED, 0) == \
+        mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_flags(A16, A16B, A16, 5, 1, 1, 4, 64, A16, 0, 4, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_qlinear_flags(A16, A16B, A16, 3, 1, 1, 4, 64, A16, 0, mpw.X_READY | mpw.Y_UNSHARED, 0) == \
+        mpw.MPW_E_UNSUPPORTED_BITS
 
 
 def test_binding_rejects_x_ready_with_workspace():
@@ -149,6 +155,8 @@ def test_binding_rejects_x_ready_with_workspace():
     s = torch.ones((4,), dtype=torch.float32)
     with pytest.raises(ValueError):
         mpw.qlinear(x, p, s, 5, x_ready=True, use_workspace=True)
+    with pytest.raises(ValueError):
+        mpw.qlinear(x, p, s, 5, y_unshared=True)
 
 
 def test_qlinear_ws_validation():

@@ -183,3 +183,65 @@ def test_recipe_run_with_aliased_slots(mpw, norm):
             y_ref, bound = (oracle.qlinear_rms_ref if nrm else oracle.qlinear_ref)(x, q, s)
             assert oracle.check_qlinear(got.float().cpu().numpy(), y_ref, bound).all(), r
     assert mpw.device_error() == 0
+
+
+@pytest.mark.parametrize("layout", ["paired", "canonical"])
+def test_unshared_outputs_then_an_unflagged_reader(mpw, layout):
+    """A and E unflagged; B and C flagged x_ready + y_unshared (inputs written
+    before E, distinct outputs), so they write y without waiting; F,
+    unflagged, reads B's output and must see it complete."""
+    import torch
+
+    rng = np.random.default_rng(515)
+    K0, NA = 5120, 6144
+    shapes = [(NA, K0, 6), (1024, K0, 5), (4096, NA, 8), (4096, K0, 7), (2048, 4096, 6)]
+    mats = [_matrix(mpw, rng, N, K, b, layout, n_rows=None if i == 0 else 254) for i, (N, K, b) in
+            enumerate(shapes)]
+    x0 = torch.empty((1, K0), dtype=torch.bfloat16, device="cuda")
+    ys = [torch.empty((1, N), dtype=torch.bfloat16, device="cuda") for N, _, _ in shapes]
+    yf = torch.empty((1, 2048), dtype=torch.bfloat16, device="cuda")
+
+    def launch():
+        (_, _, pa, sa, _), (_, _, pe, se, _), (_, _, pb, sb, _), (_, _, pc, sc, _), (_, _, pf, sf, _) = mats
+        mpw.qlinear(x0, pa, sa, 6, y=ys[0], layout=layout)                                  # A
+        mpw.qlinear(x0, pe, se, 5, y=ys[1], layout=layout)                                  # E
+        mpw.qlinear(ys[0], pb, sb, 8, y=ys[2], layout=layout, x_ready=True, y_unshared=True)  # B
+        mpw.qlinear(x0, pc, sc, 7, y=ys[3], layout=layout, x_ready=True, y_unshared=True)     # C
+        mpw.qlinear(ys[2][:, :4096], pf, sf, 6, y=yf, layout=layout)                        # F
+
+    def check(x_in):
+        xin = x_in.float().cpu().numpy()
+        a = ys[0].float().cpu().numpy()
+        bout = ys[2].float().cpu().numpy()
+        for (q, s, _, _, rows), got, xx in zip(mats, (a, ys[1], ys[2], ys[3], yf),
+                                               (xin, xin, a, xin, bout)):
+            g = got if isinstance(got, np.ndarray) else got.float().cpu().numpy()
+            y_ref, bound = oracle.qlinear_ref(xx, q, s)
+            assert oracle.check_qlinear(g[:, rows], y_ref, bound).all()
+
+    for r in range(10):
+        x_in = workloads.gen_x(1, K0, seed=600 + r).cuda()
+        for t in ys:
+            t.zero_()
+        x0.copy_(x_in)
+        launch()
+        torch.cuda.synchronize()
+        check(x_in)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        launch()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            ys[2].zero_()
+            launch()
+    torch.cuda.current_stream().wait_stream(s)
+    for r in range(10):
+        x_in = workloads.gen_x(1, K0, seed=650 + r).cuda()
+        x0.copy_(x_in)
+        g.replay()
+        torch.cuda.synchronize()
+        check(x_in)
+    del g
+    assert mpw.device_error() == 0
