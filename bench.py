@@ -367,6 +367,31 @@ def measure_prefill(mpw, pk, reps=10, layout="canonical"):
     return out
 
 
+def measure_allocator(mpw, reps=20):
+    """Host time of the water-filling bit allocator over the recipe stack's 448
+    matrix shapes (synthetic log-normal sensitivities), at the byte budget of a
+    5.7-bit mean, in both modes."""
+    import numpy as np
+
+    import workloads as wl
+
+    shapes = [(N, K) for _, _, N, K in wl.recipe_shapes()]
+    sens = np.exp(np.random.default_rng(2).normal(0.0, 1.5, size=len(shapes)))
+    params = sum(N * K for N, K in shapes)
+    budget = int(params * 5.7 / 8)
+    out = []
+    for mode in ("native", "full"):
+        mpw.allocate_bits(sens, shapes, budget, mode)
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            bits, total = mpw.allocate_bits(sens, shapes, budget, mode)
+        us = (time.perf_counter() - t0) / reps * 1e6
+        out.append({"mode": mode, "matrices": len(shapes), "budget_bytes": budget, "us": round(us, 1),
+                    "mean_bits": round(sum(b * N * K for b, (N, K) in zip(bits, shapes)) / params, 3),
+                    "bytes": total})
+    return out
+
+
 def measure_recipe(mpw, pk, steps=10, warmup=3, layout="canonical"):
     """448-matrix mixed-bit decode pass (M = 1) captured in one CUDA graph."""
     import torch
@@ -646,6 +671,7 @@ def main(argv=None):
             torch.cuda.empty_cache()
         extras["mlp27b"] = mlp
         extras["prefill"] = measure_prefill(mpw, pk, layout=lay)
+        extras["allocator"] = measure_allocator(mpw)
         extras["recipe"] = measure_recipe(mpw, pk, layout=lay)
 
     # ---- e2e: the public call with host buffers ----

@@ -293,6 +293,36 @@ MPW_API mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count,
                                      void* workspace, size_t workspace_bytes, mpw_stream_t stream);
 
 /*
+ * mpw_allocate_bits -- per-matrix bit widths under a byte budget.
+ * Pages: DynaQuant "Step 2: bit allocation" (water filling over a max-heap of
+ * marginal bit upgrades: each step raises one matrix to its next level, by
+ * quality gain per byte of cost; hardware-native {4, 8, 16} or full 4..16).
+ * The gain and the cost are this library's readings: the loss of a matrix at
+ * b bits is sens / (2^(b-1) - 1)^2 (zero at 16 bits, the unquantized bf16
+ * matrix), its cost the bytes it is stored in here (N * mpw_packed_row_bytes
+ * + 4 * N for the scales; 2 * N * K at 16 bits).  Every matrix starts at 4
+ * bits; upgrades are taken by gain / extra bytes (fp64), ties to the lower
+ * index, and one that no longer fits is dropped while the others go on.
+ *   sens    host, double [count]: per-matrix sensitivity, finite and >= 0.
+ *   N, K    host, int64 [count]: output rows and inputs of each matrix, in
+ *           1 .. 2^31 - 1.
+ *   budget  bytes for all matrices together.
+ *   mode    MPW_ALLOC_NATIVE or MPW_ALLOC_FULL.
+ *   bits    host, int32 [count], written: 4..16 (16 = keep bf16).
+ *   total   host, nullable: receives the bytes of the allocation.
+ * Runs on the host (no device work, no stream).  Null pointers, count outside
+ * 1 .. 2^24, a bad mode or size, a negative or non-finite sensitivity, or a
+ * budget below the cost of 4 bits everywhere: MPW_E_INVALID_ARG, nothing
+ * written.
+ */
+typedef enum mpw_alloc_mode {
+  MPW_ALLOC_NATIVE = 0, /* {4, 8, 16} */
+  MPW_ALLOC_FULL = 1    /* {4, 5, ..., 16} */
+} mpw_alloc_mode;
+MPW_API mpw_status mpw_allocate_bits(const double* sens, const int64_t* N, const int64_t* K, int64_t count,
+                                     uint64_t budget, int mode, int32_t* bits, uint64_t* total);
+
+/*
  * mpw_qlinear_noalloc -- the decode linear (M <= 32) on the stream-K kernel,
  * with its workspace taken from a fixed array inside the library instead of
  * from the caller, so that the call allocates no memory of any kind.

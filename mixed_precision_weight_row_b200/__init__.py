@@ -17,7 +17,7 @@ from dataclasses import dataclass
 
 __all__ = [
     "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
-    "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str",
+    "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str", "allocate_bits",
     "LAYOUTS", "workspace", "qlinear_workspace_bytes",
 ]
 
@@ -96,6 +96,8 @@ def _load():
     L.mpw_qlinear_ws.restype = c_int
     L.mpw_qlinear_flags.argtypes = [vp, vp, vp, c_int, c_int, i64, i64, i64, vp, c_int, ctypes.c_uint, vp]
     L.mpw_qlinear_flags.restype = c_int
+    L.mpw_allocate_bits.argtypes = [vp, vp, vp, i64, ctypes.c_uint64, c_int, vp, vp]
+    L.mpw_allocate_bits.restype = c_int
     L.mpw_recipe_workspace_bytes.argtypes = [ctypes.POINTER(_Linear), i64, i64]
     L.mpw_recipe_workspace_bytes.restype = ctypes.c_size_t
     L.mpw_recipe_run_ws.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp,
@@ -304,6 +306,29 @@ def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: st
                               M, N, K, y.data_ptr(), PATHS[path], None if ws is None else ws.data_ptr(),
                               ws_bytes, _stream(stream)), "mpw_qlinear")
     return y
+
+
+ALLOC_MODES = {"native": 0, "full": 1}
+
+
+def allocate_bits(sensitivity, shapes, budget_bytes: int, mode: str = "full"):
+    """Per-matrix bit widths under a byte budget (mpw_allocate_bits, host
+    only): sensitivity per matrix, shapes as (N, K) pairs; returns (bits,
+    total bytes)."""
+    import numpy as np
+
+    sens = np.ascontiguousarray(sensitivity, dtype=np.float64)
+    sh = np.ascontiguousarray(shapes, dtype=np.int64).reshape(-1, 2)
+    if sens.ndim != 1 or sens.shape[0] != sh.shape[0]:
+        raise ValueError("one sensitivity per (N, K) shape")
+    n_rows = np.ascontiguousarray(sh[:, 0])
+    k_cols = np.ascontiguousarray(sh[:, 1])
+    bits = np.zeros(sens.shape[0], dtype=np.int32)
+    total = ctypes.c_uint64(0)
+    _check(lib.mpw_allocate_bits(sens.ctypes.data, n_rows.ctypes.data, k_cols.ctypes.data, sens.shape[0],
+                                 int(budget_bytes), ALLOC_MODES[mode], bits.ctypes.data, ctypes.byref(total)),
+           "mpw_allocate_bits")
+    return bits.tolist(), int(total.value)
 
 
 @dataclass

@@ -95,3 +95,86 @@ ORIG_PACK_PAIRED = oq.pack_paired
 def test_planted_mistake_is_caught(name, monkeypatch):
     MUTANTS[name](monkeypatch)
     assert _run_pins() > 0, f"mutant {name} passed every pin"
+
+
+# ---------------------------------------------------------------------------
+# the bit allocator (oracle/alloc.py)
+# ---------------------------------------------------------------------------
+
+import heapq  # noqa: E402
+
+import oracle.alloc as oa  # noqa: E402
+from tests import test_allocator as apins  # noqa: E402
+
+ORIG_ALLOCATE = oa.allocate
+
+
+def _run_alloc_pins():
+    failures = 0
+    checks = [apins.test_matrix_bytes_matches_the_packed_format, apins.test_loss_model_follows_the_quantizer,
+              apins.test_end_points]
+    checks += [lambda m=m: apins.test_filling_states_are_optimal_for_their_budget(m) for m in ("native", "full")]
+    checks += [lambda m=m: apins.test_filling_leaves_no_upgrade_that_fits(m) for m in ("native", "full")]
+    checks += [lambda m=m: apins.test_filling_contains_the_largest_prefix_that_fits(m) for m in ("native", "full")]
+    checks += [lambda m=m: apins.test_prefix_states_are_optimal_by_exhaustive_search(m) for m in ("native",)]
+    for c in checks:
+        try:
+            c()
+        except (AssertionError, ValueError, IndexError, ZeroDivisionError):
+            failures += 1
+    return failures
+
+
+def _allocate_with(priority=lambda gain, extra: gain / extra, stop_at_first_drop=False):
+    def allocate(sens, shapes, budget, mode="full"):
+        lv = oa.step_levels(mode)
+        level = [0] * len(shapes)
+        spent = sum(oa.matrix_bytes(N, K, lv[0]) for N, K in shapes)
+        if spent > budget:
+            raise ValueError("budget")
+        heap = []
+
+        def push(i):
+            if level[i] + 1 < len(lv):
+                N, K = shapes[i]
+                b0, b1 = lv[level[i]], lv[level[i] + 1]
+                gain = oa.distortion(sens[i], b0) - oa.distortion(sens[i], b1)
+                extra = oa.matrix_bytes(N, K, b1) - oa.matrix_bytes(N, K, b0)
+                heapq.heappush(heap, (-(float("inf") if extra <= 0 else priority(gain, extra)), i, extra))
+
+        for i in range(len(shapes)):
+            push(i)
+        while heap:
+            _, i, extra = heapq.heappop(heap)
+            if spent + extra > budget:
+                if stop_at_first_drop:
+                    break
+                continue
+            spent += extra
+            level[i] += 1
+            push(i)
+        return [lv[l] for l in level], spent
+    return allocate
+
+
+ALLOC_MUTANTS = {
+    "priority_is_gain_not_gain_per_byte": lambda mp: mp.setattr(oa, "allocate", _allocate_with(lambda g, e: g)),
+    "priority_is_bytes_per_gain": lambda mp: mp.setattr(oa, "allocate", _allocate_with(lambda g, e: e / g if g else 0)),
+    "filling_stops_at_first_misfit": lambda mp: mp.setattr(oa, "allocate", _allocate_with(stop_at_first_drop=True)),
+    "loss_not_squared": lambda mp: mp.setattr(oa, "distortion",
+                                              lambda s, b: 0.0 if b == 16 else s / float(2 ** (b - 1) - 1)),
+    "bf16_costed_as_packed_codes": lambda mp: mp.setattr(
+        oa, "matrix_bytes",
+        lambda N, K, b: N * (16 * ((K * b + 127) // 128)) + 4 * N),
+}
+
+
+def test_unmutated_allocator_oracle_passes_its_pins():
+    assert oa.allocate is ORIG_ALLOCATE
+    assert _run_alloc_pins() == 0
+
+
+@pytest.mark.parametrize("name", sorted(ALLOC_MUTANTS))
+def test_planted_allocator_mistake_is_caught(name, monkeypatch):
+    ALLOC_MUTANTS[name](monkeypatch)
+    assert _run_alloc_pins() > 0, name
