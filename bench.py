@@ -683,7 +683,7 @@ def main(argv=None):
     e2e["value"] = world * e2e["value"]
 
     traffic = profile_traffic(f"gemv_tma_decode_b6_m1_{lay}.json", TMA_GEMV_SOURCES)
-    roof = {"bound": "hbm", "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,false,{str(lay == 'paired').lower()}>",
+    roof = {"bound": "hbm", "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,0,{str(lay == 'paired').lower()}>",
             "achieved": round(achieved, 1),
             "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
             "traffic": traffic, "alg_bytes_per_launch": alg_bytes,

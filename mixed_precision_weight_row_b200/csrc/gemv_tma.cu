@@ -148,21 +148,24 @@ constexpr int dec_parts() {
 }
 
 // Paired rows with one part and one token tile fit in 64 registers (56 for
-// b <= 5): six or
-// seven CTAs per SM; the rms-scaled variant keeps eight sums of squares more
-// and stays at four.
-template <int B, int NT, bool NORM, bool PAIRED>
+// b <= 5): six or seven CTAs per SM; the rms-scaled variant for one token
+// needs a few more (five CTAs), the one for up to eight tokens keeps eight
+// sums of squares and stays at four.
+template <int B, int NT, int NSQ, bool PAIRED>
 constexpr int min_ctas_for() {
-  return PAIRED && dec_parts<B, PAIRED>() == 1 && NT == 1 ? (NORM ? 4 : 6) : min_ctas<B, NT>();
+  return PAIRED && dec_parts<B, PAIRED>() == 1 && NT == 1 ? (NSQ > 1 ? 4 : (NSQ == 1 ? 5 : 6)) : min_ctas<B, NT>();
 }
 
-template <int B, int NT, bool NORM, bool PAIRED>
-__global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, NORM, PAIRED>())
+// NSQ: 0 = plain input; 1 or kNormMaxM = rms-scaled input for up to that
+// many tokens (sums of squares kept per token).
+template <int B, int NT, int NSQ, bool PAIRED>
+__global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, NSQ, PAIRED>())
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                 int M, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
                 int flags, int32_t* err) {
   constexpr int P = dec_parts<B, PAIRED>();
-  constexpr int NS = NORM ? kNormMaxM : 1;
+  constexpr bool NORM = NSQ > 0;
+  constexpr int NS = NSQ > 0 ? NSQ : 1;
   constexpr uint32_t kWChunk = 256u * B;        // 16 rows x 16*B bytes
   const uint32_t x_chunk = 256u * M;            // M tokens x 128 bf16
   const uint32_t w_part = kSC * kWChunk;
@@ -499,7 +502,7 @@ int cluster_size(int tiles, int chunks, int num_sms) {
   return best;
 }
 
-template <int B, int NT, bool NORM, bool PAIRED>
+template <int B, int NT, int NSQ, bool PAIRED>
 cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
                     uint16_t* y, bool pdl, int flags, int32_t* err, cudaStream_t stream) {
   auto encode = tensor_map_encoder();
@@ -551,14 +554,14 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = gemv_tma_kernel<B, NT, NORM, PAIRED>;
+  auto kern = gemv_tma_kernel<B, NT, NSQ, PAIRED>;
   const int tiles = (N + 15) / 16;
   const int kc = cluster_size(tiles, chunks, device_info().num_sms);
   const int per_cta = ((chunks + kc - 1) / kc + kSC - 1) / kSC;
   // resident CTAs per SM that registers and static shared memory allow
   static const int ctas_by_regs = [] {
     int n = 0;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tma_kernel<B, NT, NORM, PAIRED>, kThreads, 0) ==
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tma_kernel<B, NT, NSQ, PAIRED>, kThreads, 0) ==
                    cudaSuccess
                ? n
                : 0;
@@ -594,10 +597,11 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
 template <int B, bool PAIRED>
 cudaError_t tma_bits(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
                      uint16_t* y, bool norm, bool pdl, int flags, int32_t* err, cudaStream_t stream) {
-  if (norm) return run_tma<B, 1, true, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);  // M <= 8
-  if (M <= 8) return run_tma<B, 1, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
-  if (M <= 16) return run_tma<B, 2, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
-  return run_tma<B, 4, false, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  if (norm && M == 1) return run_tma<B, 1, 1, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  if (norm) return run_tma<B, 1, kNormMaxM, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  if (M <= 8) return run_tma<B, 1, 0, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  if (M <= 16) return run_tma<B, 2, 0, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  return run_tma<B, 4, 0, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
 }
 
 template <bool PAIRED>

@@ -81,8 +81,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t
   }
 }
 
-// Orders this thread's generic-proxy accesses to shared memory with later
-// async-proxy (TMA, tcgen05) accesses of the same memory.
 // Programmatic dependent launch: waits until the preceding grid in the stream
 // has completed (its memory visible), then lets the next grid launch.  When
 // every kernel releases its dependents only after such a wait, a kernel that
@@ -92,6 +90,8 @@ __device__ __forceinline__ void grid_dep_wait_then_release() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Orders this thread's generic-proxy accesses to shared memory with later
+// async-proxy (TMA, tcgen05) accesses of the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
