@@ -267,6 +267,30 @@ def measure_decode(mpw, pool, b, M, K, N, steps, warmup, world=1, x=None, layout
     return out
 
 
+def measure_cold_launch(mpw, pool, x, b, N, layout, l2_bytes, reps=7):
+    """One decode launch alone, after a write larger than L2 has flushed it:
+    CUDA events around the single launch, median of `reps`."""
+    import torch
+
+    flush = torch.empty(int(2 * l2_bytes), dtype=torch.uint8, device="cuda")
+    y = torch.empty((x.shape[0], N), dtype=torch.bfloat16, device="cuda")
+    times = []
+    for r in range(reps):
+        i = r % pool.P
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mpw.qlinear(x, pool.packed[i], pool.scales[i], b, y=y, layout=layout)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    us = sorted(times)[len(times) // 2]
+    del flush
+    return {"us": round(us, 3), "weight_GBps": round(pool.bytes_each / (us * 1e3), 1),
+            "note": "median of single launches after an L2 flush, events around the launch"}
+
+
 def measure_quantize(mpw, W_gpu, b, steps, warmup, l2_bytes):
     import torch
 
@@ -623,6 +647,7 @@ def main(argv=None):
         extras["dependent_chain"] = {"us_per_launch": round(r["us_per_launch"], 4),
                                      "weight_GBps": round(r["weight_GBps"], 1),
                                      "pct_hbm": round(100.0 * r["alg_GBps"] / pk["hbm_gbs"], 2)}
+        extras["cold_single_launch"] = measure_cold_launch(mpw, pool, x1, HEADLINE_BITS, N, lay, l2)
     if rank == 0 and not args.quick:
         sweep = []
         for b in DECODE_BITS:
