@@ -160,15 +160,22 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(v, world):
+def max_over_ranks(v, world, device="cuda"):
+    """The largest v over the ranks (every rank gets it)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(world, units_per_rank_step, max_ms_per_step):
+    """Units per second of the whole job: every rank processes the same units
+    per step (weak scaling) and the slowest rank sets the time."""
+    return world * units_per_rank_step / (max_ms_per_step * 1e-3)
 
 
 # ----------------------------------------------------------------------------
@@ -313,10 +320,11 @@ def measure_quantize(mpw, W_gpu, b, steps, warmup, l2_bytes):
             "weights_per_s": N * K / (per * 1e-6), "copies": copies}
 
 
-def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup, pool_n, layout="canonical"):
+def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup, pool_n, layout="canonical",
+                world=1):
     """Same metric through the public call with host buffers: each step copies
     pool_n packed matrices and x host->device, runs the GEMV on each and reads
-    y back to the host."""
+    y back to the host.  Whole-job GB/s over `world` ranks (slowest rank)."""
     import torch
 
     dp = [torch.empty_like(packed_host, device="cuda") for _ in range(2)]
@@ -337,6 +345,8 @@ def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -344,9 +354,10 @@ def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup
         step()
     e1.record()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
     wbytes = pool_n * (packed_host.numel() + scales_host.numel() * 4)
-    return {"value": wbytes * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+    return {"value": whole_job_rate(world, wbytes, ms / steps) / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": wbytes + x_host.numel() * 2,
             "d2h_bytes_per_step": M * N * 2, "ms_per_step": ms / steps}
 
@@ -633,11 +644,19 @@ def main(argv=None):
     launches = args.steps * pool.P
     ms_per_step = ms / args.steps
     weight_bytes_per_step = pool.P * pool.bytes_each
-    value = world * weight_bytes_per_step / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_rate(world, weight_bytes_per_step, ms_per_step) / 1e9
     us_launch = ms * 1e3 / launches
     alg_bytes = pool.bytes_each + K * 2 + N * 2
     achieved = alg_bytes / (us_launch * 1e-6) / 1e9
 
+    # ---- e2e: the public call with host buffers (every rank; collectives) ----
+    packed_h = pool.packed[0].cpu().pin_memory()
+    scales_h = pool.scales[0].cpu().pin_memory()
+    x_h = x1.cpu().pin_memory()
+    e2e = measure_e2e(mpw, packed_h, scales_h, x_h, HEADLINE_BITS, 1, N, K,
+                      max(3, min(args.steps, 10)), 3, pool.P, layout=lay, world=world)
+
+    # rank 0 alone from here on: no collective until the end
     extras = {}
     if rank == 0:
         # the same launches, each one waiting for its predecessor before it
@@ -698,14 +717,6 @@ def main(argv=None):
         extras["prefill"] = measure_prefill(mpw, pk, layout=lay)
         extras["allocator"] = measure_allocator(mpw)
         extras["recipe"] = measure_recipe(mpw, pk, layout=lay)
-
-    # ---- e2e: the public call with host buffers ----
-    packed_h = pool.packed[0].cpu().pin_memory()
-    scales_h = pool.scales[0].cpu().pin_memory()
-    x_h = x1.cpu().pin_memory()
-    e2e = measure_e2e(mpw, packed_h, scales_h, x_h, HEADLINE_BITS, 1, N, K,
-                      max(3, min(args.steps, 10)), 3, pool.P, layout=lay)
-    e2e["value"] = world * e2e["value"]
 
     traffic = profile_traffic(f"gemv_tma_decode_b6_m1_{lay}.json", TMA_GEMV_SOURCES)
     roof = {"bound": "hbm", "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,0,{str(lay == 'paired').lower()}>",
