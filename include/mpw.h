@@ -282,6 +282,15 @@ MPW_API mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count,
                           uint16_t* const* slots, int64_t num_slots, int64_t M,
                           mpw_stream_t stream);
 
+/*
+ * mpw_recipe_plan -- the flags mpw_recipe_run launches each linear with
+ * (0, MPW_QLINEAR_X_READY, or MPW_QLINEAR_X_READY | MPW_QLINEAR_Y_UNSHARED),
+ * written to flags[count] (host memory), from the same arguments (validated
+ * alike; slot pointers are compared, never dereferenced).  Host only.
+ */
+MPW_API mpw_status mpw_recipe_plan(const mpw_linear* layers, int64_t count, uint16_t* const* slots,
+                                   int64_t num_slots, int64_t M, uint32_t* flags);
+
 /* Workspace bytes for mpw_recipe_run_ws over these layers (the largest any
  * one of them needs). */
 MPW_API size_t mpw_recipe_workspace_bytes(const mpw_linear* layers, int64_t count, int64_t M);

@@ -18,6 +18,7 @@ from dataclasses import dataclass
 __all__ = [
     "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
     "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str", "allocate_bits",
+    "recipe_plan",
     "LAYOUTS", "workspace", "qlinear_workspace_bytes",
 ]
 
@@ -98,6 +99,9 @@ def _load():
     L.mpw_qlinear_flags.restype = c_int
     L.mpw_allocate_bits.argtypes = [vp, vp, vp, i64, ctypes.c_uint64, c_int, vp, vp]
     L.mpw_allocate_bits.restype = c_int
+    L.mpw_recipe_plan.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64,
+                                  ctypes.POINTER(ctypes.c_uint32)]
+    L.mpw_recipe_plan.restype = c_int
     L.mpw_recipe_workspace_bytes.argtypes = [ctypes.POINTER(_Linear), i64, i64]
     L.mpw_recipe_workspace_bytes.restype = ctypes.c_size_t
     L.mpw_recipe_run_ws.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp,
@@ -343,6 +347,19 @@ class Linear:
     out_slot: int
     norm_input: bool = False
     layout: str = "canonical"
+
+
+def recipe_plan(layers, slots, M: int):
+    """The MPW_QLINEAR_* flags recipe_run launches each linear with (host
+    only; slot addresses are compared, never read)."""
+    arr = (_Linear * len(layers))()
+    for i, L in enumerate(layers):
+        arr[i] = _Linear(L.packed.data_ptr(), L.scales.data_ptr(), int(L.N), int(L.K), int(L.bits),
+                         int(L.in_slot), int(L.out_slot), int(bool(L.norm_input)), LAYOUTS[L.layout], 0)
+    ptrs = (ctypes.c_void_p * len(slots))(*[s.data_ptr() for s in slots])
+    flags = (ctypes.c_uint32 * len(layers))()
+    _check(lib.mpw_recipe_plan(arr, len(layers), ptrs, len(slots), int(M), flags), "mpw_recipe_plan")
+    return list(flags)
 
 
 def recipe_run(layers, slots, M: int, stream=None, use_workspace: bool = False):

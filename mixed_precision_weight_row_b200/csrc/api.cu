@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <vector>
 
 #include "mpw.h"
 #include "mpw_internal.h"
@@ -262,6 +263,41 @@ mpw_status recipe_check(const mpw_linear* layers, int64_t count, uint16_t* const
   return MPW_OK;
 }
 
+// The MPW_QLINEAR_* flags each linear of a recipe run is launched with.  A
+// linear whose input was written neither by the linear before the current
+// run of x-ready linears nor by one inside it joins the run (X_READY): k and
+// v after q, up after gate; when its output is also neither read nor written
+// by the run and that linear, it writes it without waiting (Y_UNSHARED).
+// Inputs and outputs are compared as byte ranges, so slots that alias are
+// safe.  The first linear follows whatever the caller launched before: never.
+void recipe_flags(const mpw_linear* layers, int64_t count, uint16_t* const* slots, int64_t M, uint32_t* flags) {
+  constexpr int kRunMax = 8;
+  // inputs and outputs of the run and of the linear before it
+  uintptr_t in_lo[kRunMax], in_hi[kRunMax], out_lo[kRunMax], out_hi[kRunMax];
+  int nrun = 0;
+  auto overlaps = [&](const uintptr_t* lo, const uintptr_t* hi, uintptr_t a, uintptr_t b) {
+    for (int r = 0; r < nrun; ++r)
+      if (a < hi[r] && lo[r] < b) return true;
+    return false;
+  };
+  for (int64_t i = 0; i < count; ++i) {
+    const mpw_linear& L = layers[i];
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(slots[L.in_slot]);
+    const uintptr_t xb = xa + static_cast<uintptr_t>(M * L.K) * 2u;
+    const uintptr_t ya = reinterpret_cast<uintptr_t>(slots[L.out_slot]);
+    const uintptr_t yb = ya + static_cast<uintptr_t>(M * L.N) * 2u;
+    const bool xr = i > 0 && nrun < kRunMax && !overlaps(out_lo, out_hi, xa, xb);
+    const bool yf = xr && !overlaps(out_lo, out_hi, ya, yb) && !overlaps(in_lo, in_hi, ya, yb);
+    if (!xr) nrun = 0;
+    in_lo[nrun] = xa;
+    in_hi[nrun] = xb;
+    out_lo[nrun] = ya;
+    out_hi[nrun] = yb;
+    ++nrun;
+    flags[i] = (xr ? kQlinearXReady : 0u) | (yf ? kQlinearYFree : 0u);
+  }
+}
+
 size_t recipe_ws_bytes(const mpw_linear* layers, int64_t count, int64_t M) {
   size_t b = 0;
   for (int64_t i = 0; i < count; ++i) {
@@ -289,44 +325,24 @@ mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count, uint16_t* 
     if (!aligned(workspace, 16)) return MPW_E_MISALIGNED;
     if (workspace_bytes < recipe_ws_bytes(layers, count, M)) return MPW_E_INVALID_ARG;
   }
+  std::vector<uint32_t> flags(static_cast<size_t>(count));
+  recipe_flags(layers, count, slots, M, flags.data());
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  auto run = [&](int64_t i, cudaStream_t st, unsigned qflags) {
-    const mpw_linear& L = layers[i];
-    return launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, L.layout, M, L.N, L.K, slots[L.out_slot],
-                       L.norm_input != 0, workspace, workspace_bytes, st, qflags);
-  };
-  // A linear whose input was written neither by the linear before the
-  // current run of x-ready linears nor by one inside it joins the run
-  // (MPW_QLINEAR_X_READY): k and v after q, up after gate; when its output is
-  // also neither read nor written by the run and that linear, it writes it
-  // without waiting (MPW_QLINEAR_Y_UNSHARED).  Inputs and outputs are
-  // compared as byte ranges, so slots that alias are safe.  The first linear
-  // follows whatever the caller launched before: never.
-  constexpr int kRunMax = 8;
-  // inputs and outputs of the run and of the linear before it
-  uintptr_t in_lo[kRunMax], in_hi[kRunMax], out_lo[kRunMax], out_hi[kRunMax];
-  int nrun = 0;
-  auto overlaps = [&](const uintptr_t* lo, const uintptr_t* hi, uintptr_t a, uintptr_t b) {
-    for (int r = 0; r < nrun; ++r)
-      if (a < hi[r] && lo[r] < b) return true;
-    return false;
-  };
   for (int64_t i = 0; i < count; ++i) {
     const mpw_linear& L = layers[i];
-    const uintptr_t xa = reinterpret_cast<uintptr_t>(slots[L.in_slot]);
-    const uintptr_t xb = xa + static_cast<uintptr_t>(M * L.K) * 2u;
-    const uintptr_t ya = reinterpret_cast<uintptr_t>(slots[L.out_slot]);
-    const uintptr_t yb = ya + static_cast<uintptr_t>(M * L.N) * 2u;
-    const bool xr = i > 0 && nrun < kRunMax && !overlaps(out_lo, out_hi, xa, xb);
-    const bool yf = xr && !overlaps(out_lo, out_hi, ya, yb) && !overlaps(in_lo, in_hi, ya, yb);
-    if (!xr) nrun = 0;
-    in_lo[nrun] = xa;
-    in_hi[nrun] = xb;
-    out_lo[nrun] = ya;
-    out_hi[nrun] = yb;
-    ++nrun;
-    if (run(i, s, (xr ? kQlinearXReady : 0u) | (yf ? kQlinearYFree : 0u)) != cudaSuccess) return MPW_E_CUDA;
+    if (launch_gemv(slots[L.in_slot], L.packed, L.scales, L.bits, L.layout, M, L.N, L.K, slots[L.out_slot],
+                    L.norm_input != 0, workspace, workspace_bytes, s, flags[static_cast<size_t>(i)]) != cudaSuccess)
+      return MPW_E_CUDA;
   }
+  return MPW_OK;
+}
+
+mpw_status mpw_recipe_plan(const mpw_linear* layers, int64_t count, uint16_t* const* slots, int64_t num_slots,
+                           int64_t M, uint32_t* flags) {
+  if (flags == nullptr) return MPW_E_INVALID_ARG;
+  const mpw_status st = recipe_check(layers, count, slots, num_slots, M);
+  if (st != MPW_OK) return st;
+  recipe_flags(layers, count, slots, M, flags);
   return MPW_OK;
 }
 
