@@ -65,7 +65,9 @@ typedef enum mpw_status {
   MPW_E_CUDA = 4,             /* a CUDA runtime call or launch failed */
   MPW_E_NONFINITE = 5,        /* reserved: reported through the flag word */
   MPW_E_TIMEOUT = 6,          /* a device-side wait gave up (see mpw_device_error) */
-  MPW_E_SCRATCH_LIMIT = 7     /* mpw_qlinear_noalloc: the call needs more than its fixed scratch */
+  MPW_E_SCRATCH_LIMIT = 7,    /* mpw_qlinear_noalloc: the call needs more than its fixed scratch */
+  MPW_E_IO = 8,               /* mpw_file_*: the file cannot be opened, read or written */
+  MPW_E_FORMAT = 9            /* mpw_file_*: not a valid container, truncated, or a checksum differs */
 } mpw_status;
 
 /* Static English text for a status code; never NULL. */
@@ -330,6 +332,45 @@ typedef enum mpw_alloc_mode {
 } mpw_alloc_mode;
 MPW_API mpw_status mpw_allocate_bits(const double* sens, const int64_t* N, const int64_t* K, int64_t count,
                                      uint64_t budget, int mode, int32_t* bits, uint64_t* total);
+
+/*
+ * Packed-weight files (host only).
+ * Pages: DynaQuant "Status" (a packed weight format for disk storage is in
+ * progress); the format itself is this library's:
+ *   header, 32 bytes: "MPWPACK\0", u32 version (1), u32 count, u64 index
+ *     offset (32), u64 data offset;
+ *   index, 64 bytes per matrix: u64 N, u64 K, u32 bits, u32 layout, u64
+ *     packed offset, u64 packed bytes (N * mpw_packed_row_bytes(K, bits)),
+ *     u64 scales offset, u32 CRC-32 of the packed bytes, u32 CRC-32 of the
+ *     scales, u64 reserved (0);
+ *   data: each matrix's packed rows, then its fp32 scales, each at a multiple
+ *     of 64 bytes (zero fill).
+ * Little-endian throughout; CRC-32 of IEEE 802.3 (as zlib's crc32).
+ * Errors: MPW_E_INVALID_ARG (null pointer, bad count or index, bad shape or
+ * layout), MPW_E_UNSUPPORTED_BITS, MPW_E_IO (open / read / write failed),
+ * MPW_E_FORMAT (not a container of this version, an index entry out of the
+ * file, a checksum that differs).
+ */
+typedef struct mpw_file_matrix {
+  int64_t N;
+  int64_t K;
+  int32_t bits;
+  int32_t layout;          /* MPW_LAYOUT_* of the rows, as stored */
+  const uint8_t* packed;   /* host, N * mpw_packed_row_bytes(K, bits) bytes */
+  const float* scales;     /* host, N */
+} mpw_file_matrix;
+
+/* Writes `count` matrices (host buffers) to `path`, replacing the file. */
+MPW_API mpw_status mpw_file_write(const char* path, const mpw_file_matrix* matrices, int64_t count);
+/* Number of matrices in the file. */
+MPW_API mpw_status mpw_file_count(const char* path, int64_t* count);
+/* Shape, bit width and layout of matrix `index`. */
+MPW_API mpw_status mpw_file_info(const char* path, int64_t index, int64_t* N, int64_t* K, int32_t* bits,
+                                 int32_t* layout);
+/* Reads matrix `index` into host buffers of the sizes mpw_file_info implies
+ * and checks both checksums (MPW_E_FORMAT if either differs; the buffers may
+ * then hold the bytes read). */
+MPW_API mpw_status mpw_file_read(const char* path, int64_t index, uint8_t* packed, float* scales);
 
 /*
  * mpw_qlinear_noalloc -- the decode linear (M <= 32) on the stream-K kernel,

@@ -18,7 +18,7 @@ from dataclasses import dataclass
 __all__ = [
     "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
     "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str", "allocate_bits",
-    "recipe_plan",
+    "recipe_plan", "save_packed", "load_packed",
     "LAYOUTS", "workspace", "qlinear_workspace_bytes",
 ]
 
@@ -32,6 +32,8 @@ MPW_E_CUDA = 4
 MPW_E_NONFINITE = 5
 MPW_E_TIMEOUT = 6
 MPW_E_SCRATCH_LIMIT = 7
+MPW_E_IO = 8
+MPW_E_FORMAT = 9
 
 PATHS = {"auto": 0, "gemv": 1, "gemm": 2}
 # Packed layouts (mpw_layout): the canonical stream and its paired-halves
@@ -48,6 +50,17 @@ class MPWError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         super().__init__(f"{where}: {status_str(status)} (status {status})")
+
+
+class _FileMatrix(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int64),
+        ("K", ctypes.c_int64),
+        ("bits", ctypes.c_int32),
+        ("layout", ctypes.c_int32),
+        ("packed", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+    ]
 
 
 class _Linear(ctypes.Structure):
@@ -102,6 +115,15 @@ def _load():
     L.mpw_recipe_plan.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64,
                                   ctypes.POINTER(ctypes.c_uint32)]
     L.mpw_recipe_plan.restype = c_int
+    L.mpw_file_write.argtypes = [ctypes.c_char_p, ctypes.POINTER(_FileMatrix), i64]
+    L.mpw_file_write.restype = c_int
+    L.mpw_file_count.argtypes = [ctypes.c_char_p, ctypes.POINTER(i64)]
+    L.mpw_file_count.restype = c_int
+    L.mpw_file_info.argtypes = [ctypes.c_char_p, i64, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i32),
+                                ctypes.POINTER(i32)]
+    L.mpw_file_info.restype = c_int
+    L.mpw_file_read.argtypes = [ctypes.c_char_p, i64, vp, vp]
+    L.mpw_file_read.restype = c_int
     L.mpw_recipe_workspace_bytes.argtypes = [ctypes.POINTER(_Linear), i64, i64]
     L.mpw_recipe_workspace_bytes.restype = ctypes.c_size_t
     L.mpw_recipe_run_ws.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp,
@@ -347,6 +369,50 @@ class Linear:
     out_slot: int
     norm_input: bool = False
     layout: str = "canonical"
+
+
+def save_packed(path: str, matrices) -> None:
+    """Write packed matrices to a file (mpw_file_write).  ``matrices``: items
+    (packed uint8 [N, row_bytes], scales fp32 [N], bits, K, layout), tensors
+    on any device (copied to the host)."""
+    import torch
+
+    keep = []
+    arr = (_FileMatrix * len(matrices))()
+    for i, (packed, scales, bits, K, layout) in enumerate(matrices):
+        p = packed.detach().to("cpu").contiguous()
+        s_ = scales.detach().to("cpu", torch.float32).contiguous()
+        if p.dtype != torch.uint8 or p.dim() != 2 or p.shape[1] != packed_row_bytes(K, bits):
+            raise ValueError("packed rows must be uint8 [N, packed_row_bytes(K, bits)]")
+        if s_.dim() != 1 or s_.shape[0] != p.shape[0]:
+            raise ValueError("scales must have one entry per packed row")
+        keep += [p, s_]
+        arr[i] = _FileMatrix(p.shape[0], int(K), int(bits), LAYOUTS[layout], p.data_ptr(), s_.data_ptr())
+    _check(lib.mpw_file_write(os.fsencode(path), arr, len(matrices)), "mpw_file_write")
+
+
+def load_packed(path: str, device=None):
+    """Read every matrix of a file written by save_packed (mpw_file_read
+    checks the checksums): a list of dicts with packed, scales, bits, K, N,
+    layout; tensors on ``device`` (host if None)."""
+    import torch
+
+    n = ctypes.c_int64(0)
+    _check(lib.mpw_file_count(os.fsencode(path), ctypes.byref(n)), "mpw_file_count")
+    out = []
+    for i in range(n.value):
+        N, K, b, lay = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib.mpw_file_info(os.fsencode(path), i, ctypes.byref(N), ctypes.byref(K), ctypes.byref(b),
+                                 ctypes.byref(lay)), "mpw_file_info")
+        packed = torch.empty((N.value, packed_row_bytes(K.value, b.value)), dtype=torch.uint8)
+        scales = torch.empty((N.value,), dtype=torch.float32)
+        _check(lib.mpw_file_read(os.fsencode(path), i, packed.data_ptr(), scales.data_ptr()), "mpw_file_read")
+        layout = [k for k, v in LAYOUTS.items() if v == lay.value][0]
+        if device is not None:
+            packed, scales = packed.to(device), scales.to(device)
+        out.append({"packed": packed, "scales": scales, "bits": b.value, "K": K.value, "N": N.value,
+                    "layout": layout})
+    return out
 
 
 def recipe_plan(layers, slots, M: int):

@@ -113,6 +113,8 @@ const char* mpw_status_str(int status) {
     case MPW_E_NONFINITE: return "non-finite input";
     case MPW_E_TIMEOUT: return "device-side wait timed out";
     case MPW_E_SCRATCH_LIMIT: return "call needs more than the fixed scratch of mpw_qlinear_noalloc";
+    case MPW_E_IO: return "file cannot be opened, read or written";
+    case MPW_E_FORMAT: return "not a valid packed-weight file, or a checksum differs";
     default: return "unknown status";
   }
 }

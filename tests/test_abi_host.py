@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for st in range(0, 8):
+    for st in range(0, 10):
         assert mpw.status_str(st) and mpw.status_str(st) != "unknown status"
     assert mpw.status_str(99) == "unknown status"
 
