@@ -11,15 +11,21 @@ from .quant import (  # noqa: F401
     QLINEAR_REL_TOL,
     check_qlinear,
     dequantize,
+    dequantize_groups,
+    group_count,
+    group_scale_of_weight,
+    group_scales,
     pack,
     pack_paired,
     pair_halves,
     packed_row_bytes,
+    qlinear_groups_ref,
     qlinear_ref,
     qlinear_rows_ref,
     qmax,
     quality,
     quantize,
+    quantize_groups,
     quantize_pack,
     qlinear_rms_ref,
     rms_scale,

@@ -16,6 +16,10 @@ Sources (page title, section):
 * DynaQuant (zingnex forum thread), "Step 3: apply the recipe" and "Custom kernel
   architecture": one bit width per matrix, packed N-bit storage, expanded to the
   hardware format and multiplied on tensor cores; "Status": bit pack / unpack.
+* Quantization tutorial, exercises, item 1: group-wise scales (one per 128
+  weights; 32, 64, 128 and 256 compared) -- ``quantize_groups`` and friends,
+  groups of g consecutive weights along K, the last one shorter when g does
+  not divide K.  No kernel reads this variant yet.
 
 Readings taken where the pages are silent (each also listed in the design
 notes):
@@ -294,6 +298,76 @@ def qlinear_rms_ref(x, q: np.ndarray, s: np.ndarray):
 # ----------------------------------------------------------------------------
 # quality diagnostics (tutorial, "Step 2: quality metrics") -- not parity
 # ----------------------------------------------------------------------------
+
+# ----------------------------------------------------------------------------
+# group-wise scales (a format variant; the oracle comes before any kernel)
+# ----------------------------------------------------------------------------
+
+def group_count(K: int, g: int) -> int:
+    """Number of groups of g consecutive weights along a row of K."""
+    if g < 1:
+        raise ValueError("group size must be positive")
+    return -(-int(K) // int(g))
+
+
+def group_scales(W: np.ndarray, b: int, g: int) -> np.ndarray:
+    """s[n, j] = fl32(max |w_nk| / Q) over group j = weights k in
+    [j*g, min((j+1)*g, K)) of row n; a zero group takes fl32(1/Q).
+
+    Tutorial, exercise 1 ("one scale per 128 weights instead of per channel",
+    group sizes 32, 64, 128, 256 compared); the formula per group is the one
+    of "How quantization works".
+    """
+    W = np.asarray(W)
+    if W.dtype != np.float32 or W.ndim != 2:
+        raise TypeError("W must be a 2-D float32 array")
+    if not np.all(np.isfinite(W)):
+        raise ValueError("non-finite weight")
+    N, K = W.shape
+    Q = np.float32(qmax(b))
+    one = np.float32(1.0)
+    s = np.empty((N, group_count(K, g)), np.float32)
+    for j in range(s.shape[1]):
+        m = np.max(np.abs(W[:, j * g:(j + 1) * g]), axis=1).astype(np.float32)
+        with np.errstate(under="ignore"):
+            s[:, j] = np.where(m == 0, one / Q, m / Q).astype(np.float32)
+    return s
+
+
+def group_scale_of_weight(s: np.ndarray, K: int, g: int) -> np.ndarray:
+    """[N, K] array holding each weight's group scale."""
+    return np.repeat(np.asarray(s, np.float32), g, axis=1)[:, :K]
+
+
+def quantize_groups(W: np.ndarray, b: int, g: int):
+    """(q int32[N, K], s float32[N, ceil(K/g)]): every weight is coded with its
+    group's scale, q = clamp(rint(fl32(w / s_group)), -Q, Q)."""
+    s = group_scales(W, b, g)
+    sw = group_scale_of_weight(s, W.shape[1], g)
+    Q = qmax(b)
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        t = W / sw
+    r = np.rint(t)
+    r = np.where(np.isnan(r), np.float32(0), r)
+    return np.clip(r, -Q, Q).astype(np.int32), s
+
+
+def dequantize_groups(q: np.ndarray, s: np.ndarray, g: int) -> np.ndarray:
+    """float32[N, K]: fl32(q * s_group)."""
+    q = np.asarray(q)
+    return (q.astype(np.float32) * group_scale_of_weight(s, q.shape[1], g)).astype(np.float32)
+
+
+def qlinear_groups_ref(x, q: np.ndarray, s: np.ndarray, g: int):
+    """(y_ref, bound) in fp64 for y = x @ w_hat^T with w_hat = q * s_group,
+    accepted within 8e-3 * (|x| @ |w_hat|^T) + 1e-6 as for per-row scales."""
+    q = np.asarray(q)
+    x64 = np.asarray(x, dtype=np.float64)
+    w_hat = q.astype(np.float64) * group_scale_of_weight(s, q.shape[1], g).astype(np.float64)
+    y = x64 @ w_hat.T
+    bound = QLINEAR_REL_TOL * (np.abs(x64) @ np.abs(w_hat).T) + QLINEAR_ABS_TOL
+    return y, bound
+
 
 def quality(original: np.ndarray, reconstructed: np.ndarray) -> dict:
     o = np.asarray(original, np.float64).ravel()

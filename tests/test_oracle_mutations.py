@@ -178,3 +178,69 @@ def test_unmutated_allocator_oracle_passes_its_pins():
 def test_planted_allocator_mistake_is_caught(name, monkeypatch):
     ALLOC_MUTANTS[name](monkeypatch)
     assert _run_alloc_pins() > 0, name
+
+
+# ---------------------------------------------------------------------------
+# group-wise scales (oracle/quant.py)
+# ---------------------------------------------------------------------------
+
+from tests import test_oracle_groups as gpins  # noqa: E402
+
+
+def _run_group_pins():
+    failures = 0
+    checks = [lambda b=b: gpins.test_one_group_per_row_is_the_per_row_quantizer(b) for b in (4, 9)]
+    checks += [lambda b=b, g=g: gpins.test_groups_are_rows_of_the_reshaped_matrix(b, g)
+               for b in (5, 12) for g in (8, 128)]
+    checks += [lambda b=b: gpins.test_groups_match_exact_arithmetic(b) for b in (4, 11)]
+    checks += [lambda b=b: gpins.test_error_bound_per_group(b) for b in (6,)]
+    checks += [gpins.test_smaller_groups_reconstruct_better, gpins.test_group_linear_against_fraction_triple_loop]
+    for c in checks:
+        try:
+            c()
+        except (AssertionError, ValueError, IndexError):
+            failures += 1
+    return failures
+
+
+def _group_scales_with(axis_rows=False, last_from_row=False, shift=0):
+    def group_scales(W, b, g):
+        W = np.asarray(W)
+        N, K = W.shape
+        Q = np.float32(oq.qmax(b))
+        G = oq.group_count(K, g)
+        s = np.empty((N, G), np.float32)
+        for j in range(G):
+            if axis_rows:
+                blk = W[(j * g) % max(N, 1):(j * g) % max(N, 1) + g, :]
+                m = np.full(N, np.max(np.abs(blk)) if blk.size else 0, np.float32)
+            elif last_from_row and j == G - 1 and K % g:
+                m = np.max(np.abs(W), axis=1).astype(np.float32)
+            else:
+                lo = max(0, j * g + shift)
+                m = np.max(np.abs(W[:, lo:(j + 1) * g + shift]), axis=1).astype(np.float32) \
+                    if lo < K else np.zeros(N, np.float32)
+            s[:, j] = np.where(m == 0, np.float32(1) / Q, m / Q).astype(np.float32)
+        return s
+    return group_scales
+
+
+GROUP_MUTANTS = {
+    "groups_across_rows": lambda mp: _patch(mp, "group_scales", _group_scales_with(axis_rows=True)),
+    "last_partial_group_takes_the_row_max": lambda mp: _patch(mp, "group_scales",
+                                                              _group_scales_with(last_from_row=True)),
+    "group_boundaries_off_by_one": lambda mp: _patch(mp, "group_scales", _group_scales_with(shift=1)),
+    "linear_uses_the_first_group_scale_only": lambda mp: _patch(
+        mp, "group_scale_of_weight",
+        lambda s, K, g: np.repeat(np.asarray(s, np.float32)[:, :1], K, axis=1)),
+}
+
+
+def test_unmutated_group_oracle_passes_its_pins():
+    assert _run_group_pins() == 0
+
+
+@pytest.mark.parametrize("name", sorted(GROUP_MUTANTS))
+def test_planted_group_mistake_is_caught(name, monkeypatch):
+    GROUP_MUTANTS[name](monkeypatch)
+    assert _run_group_pins() > 0, name
