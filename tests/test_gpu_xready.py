@@ -6,7 +6,7 @@
 * Ordering, within the flag's contract (x written before the launch that
   precedes the run of flagged calls): A writes ya, B runs unflagged, then C
   (reading ya) and D (reading A's input) run flagged.  In eager launches and
-  in a replayed CUDA graph, with fresh inputs every round so that a stale
+  in a replayed CUDA graph, with fresh inputs every iteration so that a stale
   read would show, every output meets the oracle's bound
   |y - y_ref| <= 8e-3 * sum_k |x w_hat| + 1e-6, and the ys written by a run
   of flagged calls land in call order (the last write to a shared y wins).
