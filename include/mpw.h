@@ -30,7 +30,9 @@
  *     library never allocates, frees or retains caller memory.
  *   - Every call is asynchronous on `stream` (NULL = legacy default stream)
  *     and returns its status synchronously.  On an argument error nothing is
- *     launched.  No C++ exception crosses this boundary.
+ *     launched.  No C++ exception crosses this boundary.  Entry points marked
+ *     "host only" (mpw_allocate_bits, mpw_recipe_plan, mpw_file_*) do no
+ *     device work, take host memory and run to completion before returning.
  *   - Alignment: `packed` must be 16-byte aligned.  Everything else needs
  *     only its natural alignment, except where an entry point says otherwise.
  *   - A second, kernel-private ordering of the same bits ("paired halves",
