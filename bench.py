@@ -421,9 +421,12 @@ def measure_allocator(mpw, reps=20):
         for _ in range(reps):
             bits, total = mpw.allocate_bits(sens, shapes, budget, mode)
         us = (time.perf_counter() - t0) / reps * 1e6
+        t0 = time.perf_counter()
+        fb, fl = mpw.allocation_frontier(sens, shapes, mode)
+        us_front = (time.perf_counter() - t0) * 1e6
         out.append({"mode": mode, "matrices": len(shapes), "budget_bytes": budget, "us": round(us, 1),
                     "mean_bits": round(sum(b * N * K for b, (N, K) in zip(bits, shapes)) / params, 3),
-                    "bytes": total})
+                    "bytes": total, "frontier_points": len(fb), "frontier_us": round(us_front, 1)})
     return out
 
 

@@ -31,7 +31,7 @@
  *   - Every call is asynchronous on `stream` (NULL = legacy default stream)
  *     and returns its status synchronously.  On an argument error nothing is
  *     launched.  No C++ exception crosses this boundary.  Entry points marked
- *     "host only" (mpw_allocate_bits, mpw_recipe_plan, mpw_file_*) do no
+ *     "host only" (mpw_allocate_*, mpw_recipe_plan, mpw_file_*) do no
  *     device work, take host memory and run to completion before returning.
  *   - Alignment: `packed` must be 16-byte aligned.  Everything else needs
  *     only its natural alignment, except where an entry point says otherwise.
@@ -334,6 +334,24 @@ typedef enum mpw_alloc_mode {
 } mpw_alloc_mode;
 MPW_API mpw_status mpw_allocate_bits(const double* sens, const int64_t* N, const int64_t* K, int64_t count,
                                      uint64_t budget, int mode, int32_t* bits, uint64_t* total);
+
+/*
+ * mpw_allocate_frontier -- the trade-off curve the water filling walks
+ * (DynaQuant "Step 2": a Pareto-front allocator): the bytes and the total
+ * loss (sum of sens / (2^(b-1) - 1)^2, as for mpw_allocate_bits) after each
+ * upgrade of the filling without a budget, from 4 bits everywhere to bf16
+ * everywhere; each point is the allocation mpw_allocate_bits returns for
+ * that many bytes.  The total loss is updated by subtracting each
+ * upgrade's gain, in fp64, in that order.
+ *   sens, N, K, count, mode  as for mpw_allocate_bits.
+ *   bytes, loss  host, [max_points]: the first min(points, max_points)
+ *           points (may be NULL when max_points is 0).
+ *   n_points  receives the number of points (count * levels-above-4 + 1).
+ * Host only.  Errors as for mpw_allocate_bits (there is no budget).
+ */
+MPW_API mpw_status mpw_allocate_frontier(const double* sens, const int64_t* N, const int64_t* K, int64_t count,
+                                         int mode, uint64_t* bytes, double* loss, int64_t max_points,
+                                         int64_t* n_points);
 
 /*
  * Packed-weight files (host only).

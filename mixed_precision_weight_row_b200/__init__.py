@@ -17,7 +17,7 @@ from dataclasses import dataclass
 
 __all__ = [
     "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
-    "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str", "allocate_bits",
+    "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str", "allocate_bits", "allocation_frontier",
     "recipe_plan", "save_packed", "load_packed",
     "LAYOUTS", "workspace", "qlinear_workspace_bytes",
 ]
@@ -112,6 +112,8 @@ def _load():
     L.mpw_qlinear_flags.restype = c_int
     L.mpw_allocate_bits.argtypes = [vp, vp, vp, i64, ctypes.c_uint64, c_int, vp, vp]
     L.mpw_allocate_bits.restype = c_int
+    L.mpw_allocate_frontier.argtypes = [vp, vp, vp, i64, c_int, vp, vp, i64, ctypes.POINTER(i64)]
+    L.mpw_allocate_frontier.restype = c_int
     L.mpw_recipe_plan.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64,
                                   ctypes.POINTER(ctypes.c_uint32)]
     L.mpw_recipe_plan.restype = c_int
@@ -355,6 +357,28 @@ def allocate_bits(sensitivity, shapes, budget_bytes: int, mode: str = "full"):
                                  int(budget_bytes), ALLOC_MODES[mode], bits.ctypes.data, ctypes.byref(total)),
            "mpw_allocate_bits")
     return bits.tolist(), int(total.value)
+
+
+def allocation_frontier(sensitivity, shapes, mode: str = "full"):
+    """(bytes, total loss) after each upgrade of the unbounded water filling
+    (mpw_allocate_frontier, host only)."""
+    import numpy as np
+
+    sens = np.ascontiguousarray(sensitivity, dtype=np.float64)
+    sh = np.ascontiguousarray(shapes, dtype=np.int64).reshape(-1, 2)
+    if sens.ndim != 1 or sens.shape[0] != sh.shape[0]:
+        raise ValueError("one sensitivity per (N, K) shape")
+    n_rows = np.ascontiguousarray(sh[:, 0])
+    k_cols = np.ascontiguousarray(sh[:, 1])
+    n = ctypes.c_int64(0)
+    _check(lib.mpw_allocate_frontier(sens.ctypes.data, n_rows.ctypes.data, k_cols.ctypes.data, sens.shape[0],
+                                     ALLOC_MODES[mode], None, None, 0, ctypes.byref(n)), "mpw_allocate_frontier")
+    nbytes = np.zeros(n.value, dtype=np.uint64)
+    loss = np.zeros(n.value, dtype=np.float64)
+    _check(lib.mpw_allocate_frontier(sens.ctypes.data, n_rows.ctypes.data, k_cols.ctypes.data, sens.shape[0],
+                                     ALLOC_MODES[mode], nbytes.ctypes.data, loss.ctypes.data, n.value,
+                                     ctypes.byref(n)), "mpw_allocate_frontier")
+    return [int(v) for v in nbytes], loss.tolist()
 
 
 @dataclass

@@ -97,6 +97,42 @@ def allocate(sens, shapes, budget: int, mode: str = "full"):
     return [lv[l] for l in level], spent
 
 
+def frontier(sens, shapes, mode: str = "full"):
+    """The curve the filling walks without a budget: (bytes, total loss)
+    after each upgrade, from the lowest level everywhere to the highest.
+    The total starts as the sum of the losses in matrix order and each
+    upgrade subtracts its gain (fp64, in that order)."""
+    lv = step_levels(mode)
+    level = [0] * len(shapes)
+    spent = sum(matrix_bytes(N, K, lv[0]) for N, K in shapes)
+    total = 0.0
+    for i in range(len(shapes)):
+        total += distortion(sens[i], lv[0])
+    heap = []
+
+    def push(i):
+        if level[i] + 1 < len(lv):
+            N, K = shapes[i]
+            b0, b1 = lv[level[i]], lv[level[i] + 1]
+            gain = distortion(sens[i], b0) - distortion(sens[i], b1)
+            extra = matrix_bytes(N, K, b1) - matrix_bytes(N, K, b0)
+            prio = float("inf") if extra <= 0 else gain / extra
+            heapq.heappush(heap, (-prio, i, extra))
+
+    for i in range(len(shapes)):
+        push(i)
+    points = [(spent, total)]
+    while heap:
+        _, i, extra = heapq.heappop(heap)
+        l = level[i]
+        total -= distortion(sens[i], lv[l]) - distortion(sens[i], lv[l + 1])
+        spent += extra
+        level[i] += 1
+        push(i)
+        points.append((spent, total))
+    return points
+
+
 def exhaustive(sens, shapes, budget: int, mode: str = "full"):
     """Brute force over every assignment of levels (tiny inputs only):
     (least total distortion within the budget, its bits)."""

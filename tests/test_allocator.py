@@ -235,3 +235,64 @@ def test_allocate_bits_validation():
     assert L.mpw_allocate_bits(neg, n, k, 2, big, 1, bits, None) == mpw.MPW_E_INVALID_ARG
     zero_k = (ctypes.c_int64 * 2)(128, 0)
     assert L.mpw_allocate_bits(d, n, zero_k, 2, big, 1, bits, None) == mpw.MPW_E_INVALID_ARG
+
+
+# ---------------------------------------------------------------------------
+# the frontier the filling walks
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", ["native", "full"])
+def test_frontier_is_the_sorted_prefix_states(mode):
+    """Bytes of every frontier point are those of the ratio-sorted prefix
+    states (which exhaustive search pins), the loss is that state's total,
+    and the filling at that budget returns that state."""
+    rng = np.random.default_rng(61)
+    for trial in range(10):
+        sens, shapes = _instance(rng, 5)
+        pts = alloc.frontier(sens, shapes, mode)
+        states = _prefix_states(sens, shapes, mode)
+        assert len(pts) == len(states) == 1 + len(shapes) * (len(alloc.step_levels(mode)) - 1)
+        for (b, l), (c, bits) in zip(pts, states):
+            assert b == c
+            d = sum(alloc.distortion(s_, x) for s_, x in zip(sens, bits))
+            assert abs(l - d) <= 1e-9 * max(1.0, abs(d))
+            assert alloc.allocate(sens, shapes, b, mode)[0] == bits
+        losses = [l for _, l in pts]
+        assert all(a >= c - 1e-12 * abs(a) for a, c in zip(losses, losses[1:]))
+        assert pts[-1][1] == pytest.approx(0.0, abs=1e-12 * losses[0])
+
+
+@pytest.mark.parametrize("mode", ["native", "full"])
+def test_library_frontier_matches_oracle(mode):
+    rng = np.random.default_rng(71)
+    for trial in range(10):
+        sens, shapes = _instance(rng, int(rng.integers(1, 30)), k_mult=int(rng.choice([100, 128, 17])))
+        b_lib, l_lib = mpw.allocation_frontier(sens, shapes, mode)
+        pts = alloc.frontier(sens, shapes, mode)
+        assert b_lib == [b for b, _ in pts]
+        assert l_lib == [l for _, l in pts]          # same fp64 operations in the same order
+    shapes = [(N, K) for _, _, N, K in wl.recipe_shapes()]
+    sens = list(np.exp(np.random.default_rng(72).normal(0, 1.5, size=len(shapes))))
+    b_lib, l_lib = mpw.allocation_frontier(sens, shapes, mode)
+    pts = alloc.frontier(sens, shapes, mode)
+    assert b_lib == [b for b, _ in pts] and l_lib == [l for _, l in pts]
+
+
+def test_allocate_frontier_validation():
+    L = mpw.lib
+    d = (ctypes.c_double * 2)(1.0, 2.0)
+    n = (ctypes.c_int64 * 2)(64, 64)
+    k = (ctypes.c_int64 * 2)(128, 128)
+    cnt = ctypes.c_int64(-1)
+    assert L.mpw_allocate_frontier(d, n, k, 2, 0, None, None, 0, ctypes.byref(cnt)) == 0 and cnt.value == 5
+    assert L.mpw_allocate_frontier(d, n, k, 2, 1, None, None, 0, ctypes.byref(cnt)) == 0 and cnt.value == 25
+    assert L.mpw_allocate_frontier(d, n, k, 2, 1, None, None, 3, ctypes.byref(cnt)) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_allocate_frontier(d, n, k, 0, 1, None, None, 0, ctypes.byref(cnt)) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_allocate_frontier(d, n, k, 2, 7, None, None, 0, ctypes.byref(cnt)) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_allocate_frontier(d, n, k, 2, 1, None, None, 0, None) == mpw.MPW_E_INVALID_ARG
+    # a short buffer gets the first points and the full count
+    b3 = (ctypes.c_uint64 * 3)()
+    l3 = (ctypes.c_double * 3)()
+    assert L.mpw_allocate_frontier(d, n, k, 2, 1, b3, l3, 3, ctypes.byref(cnt)) == 0 and cnt.value == 25
+    pts = alloc.frontier([1.0, 2.0], [(64, 128), (64, 128)], "full")
+    assert [int(v) for v in b3] == [p[0] for p in pts[:3]] and list(l3) == [p[1] for p in pts[:3]]
