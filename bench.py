@@ -196,6 +196,51 @@ class Pool:
         torch.cuda.synchronize()
 
 
+# Where a code in the device error word comes from: 100 * kernel + place.
+WAIT_KERNELS = {1: "gemv_tma_kernel", 2: "gemv_tc_kernel", 3: "gemm_kernel", 4: "gemv_sk_kernel"}
+WAIT_PLACES = {1: "x producer: free x stage", 2: "x producer: last copies", 3: "producer: free stage",
+               4: "producer: last copies", 5: "consumer / MMA issuer: loaded stage",
+               6: "MMA issuer: converted weights", 7: "converter: loaded weight stage",
+               8: "converter: free tensor-memory stage", 9: "epilogue: accumulator",
+               10: "sums of squares: loaded x stage"}
+
+
+def describe_wait_code(code):
+    k, p = divmod(int(code), 100)
+    return f"{WAIT_KERNELS.get(k, f'kernel {k}')}, {WAIT_PLACES.get(p, f'place {p}')}"
+
+
+class Sections:
+    """Runs the bench's measurements one by one.  After each one the device
+    error word is read (and cleared), so that a wait that gave up is charged
+    to the section that ran it; a section that raises or sets the word is
+    recorded in `errors` and the remaining sections still run."""
+
+    def __init__(self, mpw):
+        self.mpw = mpw
+        self.errors = []
+        self.names = []
+
+    def run(self, name, fn, *args, **kw):
+        self.names.append(name)
+        result = None
+        try:
+            result = fn(*args, **kw)
+        except Exception as e:  # recorded on the JSON line instead of ending the run
+            self.errors.append({"section": name, "error": f"{type(e).__name__}: {e}"[:400]})
+        try:
+            code = self.mpw.device_error()
+        except Exception as e:
+            self.errors.append({"section": name, "error": f"device error word unreadable: {e}"[:400]})
+            return result
+        if code:
+            self.errors.append({"section": name, "device_error": code, "where": describe_wait_code(code)})
+        return result
+
+    def failed(self, name):
+        return any(e["section"] == name for e in self.errors)
+
+
 def graph_of(fn):
     import torch
 
@@ -398,7 +443,6 @@ def measure_prefill(mpw, pk, reps=10, layout="canonical"):
             del packed, scales, y
         del W
         torch.cuda.empty_cache()
-    assert mpw.device_error() == 0
     return out
 
 
@@ -626,7 +670,9 @@ def main(argv=None):
     W_np = wl.gen_weight(N, K, c["sigma"], c["w_seed"], c["outlier_frac"], c["outlier_scale"])
     W = torch.from_numpy(W_np).cuda()
 
-    # ---- headline: b = 6, M = 1 ----
+    sec = Sections(mpw)
+
+    # ---- headline: b = 6, M = 1 (every rank; collectives inside) ----
     lay = args.layout
     pool = decode_setup(mpw, W, HEADLINE_BITS, l2, lay)
     x1 = wl.gen_x(1, K, c["x_seed"]).cuda()
@@ -639,57 +685,70 @@ def main(argv=None):
             mpw.qlinear(x1, pool.packed[i], pool.scales[i], HEADLINE_BITS, y=y1[i], layout=lay, x_ready=True,
                         y_unshared=True)
 
-    g = graph_of(step)
-    with ClockSampler(uuid) as cs:
-        ms = time_graph(g, args.steps, args.warmup, world)
-    clocks = cs.summary()
-    del g
+    def headline():
+        g = graph_of(step)
+        with ClockSampler(uuid) as cs:
+            ms = time_graph(g, args.steps, args.warmup, world)
+        del g
+        return ms, cs.summary()
+
+    ms, clocks = sec.run("headline", headline) or (None, None)
     launches = args.steps * pool.P
-    ms_per_step = ms / args.steps
     weight_bytes_per_step = pool.P * pool.bytes_each
-    value = whole_job_rate(world, weight_bytes_per_step, ms_per_step) / 1e9
-    us_launch = ms * 1e3 / launches
     alg_bytes = pool.bytes_each + K * 2 + N * 2
-    achieved = alg_bytes / (us_launch * 1e-6) / 1e9
+    if ms is not None:
+        ms_per_step = ms / args.steps
+        value = whole_job_rate(world, weight_bytes_per_step, ms_per_step) / 1e9
+        us_launch = ms * 1e3 / launches
+        achieved = alg_bytes / (us_launch * 1e-6) / 1e9
+    else:
+        ms_per_step = value = us_launch = achieved = None
 
     # ---- e2e: the public call with host buffers (every rank; collectives) ----
     packed_h = pool.packed[0].cpu().pin_memory()
     scales_h = pool.scales[0].cpu().pin_memory()
     x_h = x1.cpu().pin_memory()
-    e2e = measure_e2e(mpw, packed_h, scales_h, x_h, HEADLINE_BITS, 1, N, K,
-                      max(3, min(args.steps, 10)), 3, pool.P, layout=lay, world=world)
+    e2e = sec.run("e2e", measure_e2e, mpw, packed_h, scales_h, x_h, HEADLINE_BITS, 1, N, K,
+                  max(3, min(args.steps, 10)), 3, pool.P, layout=lay, world=world)
 
     # rank 0 alone from here on: no collective until the end
     extras = {}
     if rank == 0:
         # the same launches, each one waiting for its predecessor before it
         # reads x (what a chain of dependent linears sees)
-        r = measure_decode(mpw, pool, HEADLINE_BITS, 1, K, N, max(20, args.steps // 4), 3, layout=lay,
-                           x=x1, x_ready=False)
-        extras["dependent_chain"] = {"us_per_launch": round(r["us_per_launch"], 4),
-                                     "weight_GBps": round(r["weight_GBps"], 1),
-                                     "pct_hbm": round(100.0 * r["alg_GBps"] / pk["hbm_gbs"], 2)}
-        extras["cold_single_launch"] = measure_cold_launch(mpw, pool, x1, HEADLINE_BITS, N, lay, l2)
+        r = sec.run("dependent_chain", measure_decode, mpw, pool, HEADLINE_BITS, 1, K, N,
+                    max(20, args.steps // 4), 3, layout=lay, x=x1, x_ready=False)
+        if r is not None:
+            extras["dependent_chain"] = {"us_per_launch": round(r["us_per_launch"], 4),
+                                         "weight_GBps": round(r["weight_GBps"], 1),
+                                         "pct_hbm": round(100.0 * r["alg_GBps"] / pk["hbm_gbs"], 2)}
+        extras["cold_single_launch"] = sec.run("cold_single_launch", measure_cold_launch, mpw, pool, x1,
+                                               HEADLINE_BITS, N, lay, l2)
     if rank == 0 and not args.quick:
+        def row(r, layout):
+            r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
+            r["layout"] = layout
+            return {k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()
+                    if k in ("b", "M", "layout", "us_per_launch", "weight_GBps", "alg_GBps", "pct_hbm")}
+
         sweep = []
         for b in DECODE_BITS:
-            p = pool if b == HEADLINE_BITS else decode_setup(mpw, W, b, l2, lay)
+            p = pool if b == HEADLINE_BITS else sec.run(f"decode_setup b={b}", decode_setup, mpw, W, b, l2, lay)
+            if p is None:
+                continue
             for M in DECODE_MS:
-                r = measure_decode(mpw, p, b, M, K, N, max(20, args.steps // 4), 3, layout=lay)
-                r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
-                r["layout"] = lay
-                sweep.append({k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()
-                              if k in ("b", "M", "layout", "us_per_launch", "weight_GBps", "alg_GBps",
-                                       "pct_hbm")})
+                r = sec.run(f"decode_sweep b={b} M={M}", measure_decode, mpw, p, b, M, K, N,
+                            max(20, args.steps // 4), 3, layout=lay)
+                if r is not None:
+                    sweep.append(row(r, lay))
             if lay != "canonical":
                 # the canonical rows, read directly (no re-ordering), at M = 1
-                pc = decode_setup(mpw, W, b, l2)
-                r = measure_decode(mpw, pc, b, 1, K, N, max(20, args.steps // 4), 3)
-                r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
-                r["layout"] = "canonical"
-                sweep.append({k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()
-                              if k in ("b", "M", "layout", "us_per_launch", "weight_GBps", "alg_GBps",
-                                       "pct_hbm")})
+                pc = sec.run(f"decode_setup canonical b={b}", decode_setup, mpw, W, b, l2)
+                if pc is not None:
+                    r = sec.run(f"decode_sweep canonical b={b} M=1", measure_decode, mpw, pc, b, 1, K, N,
+                                max(20, args.steps // 4), 3)
+                    if r is not None:
+                        sweep.append(row(r, "canonical"))
                 del pc
             if p is not pool:
                 del p
@@ -697,53 +756,70 @@ def main(argv=None):
         extras["decode_sweep"] = sweep
         extras["quantize_pack"] = []
         for b in (4, 6, 8, 12):
-            r = measure_quantize(mpw, W, b, 20, 3, l2)
-            r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
-            extras["quantize_pack"].append({k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()})
+            r = sec.run(f"quantize_pack b={b}", measure_quantize, mpw, W, b, 20, 3, l2)
+            if r is not None:
+                r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
+                extras["quantize_pack"].append({k: (round(v, 4) if isinstance(v, float) else v)
+                                                for k, v in r.items()})
         mlp = []
         for name, n_, k_ in wl.MLP27B["shapes"][1:]:
             Wm = wl.gen_weight_torch(n_, k_, wl.MLP27B["sigma"], 17 + n_)
             for b in wl.MLP27B["bits"]:
-                pm = decode_setup(mpw, Wm, b, l2, lay)
+                pm = sec.run(f"mlp27b setup {name} b={b}", decode_setup, mpw, Wm, b, l2, lay)
+                if pm is None:
+                    continue
                 for M in wl.MLP27B["Ms"]:
-                    r = measure_decode(mpw, pm, b, M, k_, n_, 20, 3,
-                                       x=wl.gen_x(M, k_, 1).cuda(), layout=lay)
-                    mlp.append({"shape": f"{name} {n_}x{k_}", "b": b, "M": M,
-                                "us_per_launch": round(r["us_per_launch"], 3),
-                                "weight_GBps": round(r["weight_GBps"], 1),
-                                "pct_hbm": round(100 * r["alg_GBps"] / pk["hbm_gbs"], 2)})
+                    r = sec.run(f"mlp27b {name} b={b} M={M}", measure_decode, mpw, pm, b, M, k_, n_, 20, 3,
+                                x=wl.gen_x(M, k_, 1).cuda(), layout=lay)
+                    if r is not None:
+                        mlp.append({"shape": f"{name} {n_}x{k_}", "b": b, "M": M,
+                                    "us_per_launch": round(r["us_per_launch"], 3),
+                                    "weight_GBps": round(r["weight_GBps"], 1),
+                                    "pct_hbm": round(100 * r["alg_GBps"] / pk["hbm_gbs"], 2)})
                 del pm
                 torch.cuda.empty_cache()
             del Wm
             torch.cuda.empty_cache()
         extras["mlp27b"] = mlp
-        extras["prefill"] = measure_prefill(mpw, pk, layout=lay)
-        extras["allocator"] = measure_allocator(mpw)
-        extras["recipe"] = measure_recipe(mpw, pk, layout=lay)
+        extras["prefill"] = sec.run("prefill", measure_prefill, mpw, pk, layout=lay)
+        extras["allocator"] = sec.run("allocator", measure_allocator, mpw)
+        extras["recipe"] = sec.run("recipe", measure_recipe, mpw, pk, layout=lay)
+        summary = {}
+        for p in extras.get("prefill") or []:
+            summary[f"prefill {p['shape']} b={p['b']} TFLOPs"] = p["TFLOPs"]
+        if extras.get("recipe"):
+            summary["recipe tokens_per_s"] = extras["recipe"]["tokens_per_s"]
+            summary["recipe pct_hbm"] = extras["recipe"]["pct_hbm"]
+        extras["summary"] = summary
 
     traffic = profile_traffic(f"gemv_tma_decode_b6_m1_{lay}.json", TMA_GEMV_SOURCES)
     roof = {"bound": "hbm", "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,0,{str(lay == 'paired').lower()}>",
-            "achieved": round(achieved, 1),
-            "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+            "achieved": round(achieved, 1) if achieved is not None else None,
+            "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4) if achieved is not None else None,
             "traffic": traffic, "alg_bytes_per_launch": alg_bytes,
-            "peak_source": pk["source"] + " (copy bandwidth)"}
+            "us_per_launch": round(us_launch, 4) if us_launch is not None else None,
+            "peak_source": pk["source"] + " (copy bandwidth; burst figure, kernel timed alone)"}
 
-    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+    line = {"metric": METRIC, "value": round(value, 2) if value is not None else None, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 5) if ms_per_step is not None else None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": decode_config(args, pool.P),
             "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
-            "pct_hbm_peak": round(100 * value / world / pk["hbm_gbs"], 2)}
+            "pct_hbm_peak": round(100 * value / world / pk["hbm_gbs"], 2) if value is not None else None}
     line.update(extras)
     if rank == 0 and world == 1 and not args.quick:
         line["cpu_baseline"] = cpu_baseline(seconds=10.0)
+    line["sections"] = len(sec.names)
+    line["errors"] = sec.errors
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
 
         dist.destroy_process_group()
-    return 0
+    return 0 if value is not None else 1
 
 
 if __name__ == "__main__":

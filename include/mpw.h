@@ -120,12 +120,14 @@ MPW_API mpw_status mpw_dequantize(const uint8_t* packed, const float* scales,
  *   packed, scales  as produced by mpw_quantize_pack for W [N, K].
  *   y        device, bf16 [M, N] row-major; y[m, n] is
  *            bf16_rn(s_n * sum_k x[m, k] * q[n, k]) with an fp32 accumulator.
- *   M >= 1.  M <= 32 runs the decode GEMV kernel (packed rows streamed once,
- *   unpacked in registers, mma.sync tensor cores); larger M runs the prefill
- *   GEMM on tcgen05 tensor cores with the accumulator in tensor memory.  Every
- *   code reaches the tensor cores as exact bf16 values: whole when it fits,
- *   else split into fields (256*hi + lo in the GEMM, 7-bit fields in the
- *   GEMV), each exact in bf16, so no code is ever rounded.
+ *   M >= 1.  M <= 32 runs a decode kernel (packed rows streamed once,
+ *   unpacked in registers, mma.sync or tcgen05 tensor cores); larger M runs
+ *   the prefill GEMM on tcgen05 tensor cores with the accumulator in tensor
+ *   memory.  Every code reaches the tensor cores as exact bf16 values: whole
+ *   when it has at most 9 bits, else split as lo7 + 128 * hi (lo7 = q & 127,
+ *   hi = q >> 7, arithmetic) in the GEMM and on paired rows, and into 7-bit
+ *   fields in the canonical-row decode kernels; each term is exact in bf16,
+ *   so no code is ever rounded.
  * Pages: DynaQuant "Custom kernel architecture" (packed N-bit -> registers ->
  * tensor core; 9-15 bit codes on BF16 tensor cores).
  */
@@ -406,9 +408,13 @@ MPW_API mpw_status mpw_file_read(const char* path, int64_t index, uint8_t* packe
  *     loads the library, for the life of the process.  A call whose
  *     workspace would exceed it returns MPW_E_SCRATCH_LIMIT and launches
  *     nothing; mpw_qlinear_workspace_bytes tells the size in advance.
+ *     The 27B-class gate/up matrices (17408 x 5120) at M = 32 already need
+ *     more and are refused; at M <= 8 they fit.
  *   - The first call on a device looks up the array's device address (once
  *     per device, with that device current); make that first call before any
- *     stream capture.
+ *     stream capture.  The address is kept for the life of the process, so
+ *     after cudaDeviceReset this entry point must not be called again in
+ *     that process.
  *   - Every call shares the array.  Each call clears the per-tile counters
  *     it uses (a memset on `stream`) before its kernel; the partial sums need
  *     no clearing.  Calls that overlap on the GPU (on different streams, or
@@ -423,9 +429,21 @@ MPW_API mpw_status mpw_qlinear_noalloc(const uint16_t* x, const uint8_t* packed,
 
 /*
  * mpw_device_error -- synchronises the current device, returns in *code the
- * library's device-side error word (0 = none; 1 = a bounded wait inside a
- * tensor-core kernel gave up) and clears it.  Returns MPW_E_TIMEOUT when the
- * word was set, MPW_OK otherwise.
+ * library's device-side error word and clears it.  Returns MPW_E_TIMEOUT
+ * when the word was set, MPW_OK otherwise.
+ *   0      no wait gave up since the word was last read.
+ *   other  the first bounded wait (2 s of waiting) inside a TMA / tensor-core
+ *          kernel that gave up, as 100 * kernel + place: kernel 1 = per-tile
+ *          decode, 2 = tensor-memory decode, 3 = prefill GEMM, 4 = stream-K
+ *          decode; place 1 = x producer waiting for a free stage, 2 = x
+ *          producer waiting for its last copies, 3 / 4 = the same for the
+ *          weight (or combined) producer, 5 = consumer or MMA issuer waiting
+ *          for a loaded stage, 6 = MMA issuer waiting for converted weights,
+ *          7 = converter waiting for a loaded weight stage, 8 = converter
+ *          waiting for a free tensor-memory stage, 9 = epilogue waiting for
+ *          the accumulator, 10 = sums of squares waiting for a loaded x stage.
+ *          The outputs of the call that gave up, and of calls that depend
+ *          on them, are undefined.
  */
 MPW_API mpw_status mpw_device_error(int32_t* code);
 

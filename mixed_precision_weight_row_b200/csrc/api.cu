@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -92,9 +93,19 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 int32_t* device_error_word() {
-  void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-  return static_cast<int32_t*>(p);
+  // looked up once per device (with that device current) and kept for the
+  // life of the process, like the kernels' shared-memory attributes
+  static std::atomic<int32_t*> addr[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  int32_t* a = addr[dev].load(std::memory_order_acquire);
+  if (a == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    a = static_cast<int32_t*>(p);
+    addr[dev].store(a, std::memory_order_release);
+  }
+  return a;
 }
 
 }  // namespace mpw

@@ -145,13 +145,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       int issued = 0;
       for (int kb = 0; kb < KB; ++kb) {
         const int s = kb % SX;
-        if (!ptx::mbar_wait(empty_x(s), ((kb / SX) & 1) ^ 1, err)) break;
+        if (!ptx::mbar_wait(empty_x(s), ((kb / SX) & 1) ^ 1, err, ptx::wait_code(ptx::kWaitGemm, ptx::kWaitXEmpty))) break;
         ptx::mbar_arrive_expect_tx(full_x(s), kXStageBytes);
         ptx::tma_load_2d(xs0 + s * kXStageBytes, &tmap_x, full_x(s), kb * BK, m0);
         issued = kb + 1;
       }
       // nothing may still be landing in shared memory when the CTA exits
-      for (int kb = max(0, issued - SX); kb < issued; ++kb) ptx::mbar_wait(full_x(kb % SX), (kb / SX) & 1, err);
+      for (int kb = max(0, issued - SX); kb < issued; ++kb) ptx::mbar_wait(full_x(kb % SX), (kb / SX) & 1, err, ptx::wait_code(ptx::kWaitGemm, ptx::kWaitXTail));
     }
   } else if (warp == 3) {
     // ---------------- weight producer: one TMA per block ----------------
@@ -159,13 +159,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       int issued = 0;
       for (int wb = 0; wb < WBs; ++wb) {
         const int s = wb % SW;
-        if (!ptx::mbar_wait(empty_w(s), ((wb / SW) & 1) ^ 1, err)) break;
+        if (!ptx::mbar_wait(empty_w(s), ((wb / SW) & 1) ^ 1, err, ptx::wait_code(ptx::kWaitGemm, ptx::kWaitWEmpty))) break;
         ptx::mbar_arrive_expect_tx(full_w(s), C::WSTAGE);
         ptx::tma_load_2d(ws0 + s * C::WSTAGE, &tmap_w, full_w(s), wb * 16 * B, n0);
         issued = wb + 1;
       }
       // nothing may still be landing in shared memory when the CTA exits
-      for (int wb = max(0, issued - SW); wb < issued; ++wb) ptx::mbar_wait(full_w(wb % SW), (wb / SW) & 1, err);
+      for (int wb = max(0, issued - SW); wb < issued; ++wb) ptx::mbar_wait(full_w(wb % SW), (wb / SW) & 1, err, ptx::wait_code(ptx::kWaitGemm, ptx::kWaitWTail));
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -175,8 +175,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       for (int kb = 0; kb < KB && ok; ++kb) {
         const int sx = kb % SX;
         const int wb = kb >> 1, h = kb & 1, sa = wb % SA;
-        ok = ptx::mbar_wait(full_x(sx), (kb / SX) & 1, err);
-        if (ok && h == 0) ok = ptx::mbar_wait(full_a(sa), (wb / SA) & 1, err);
+        ok = ptx::mbar_wait(full_x(sx), (kb / SX) & 1, err, ptx::wait_code(ptx::kWaitGemm, ptx::kWaitFull));
+        if (ok && h == 0) ok = ptx::mbar_wait(full_a(sa), (wb / SA) & 1, err, ptx::wait_code(ptx::kWaitGemm, ptx::kWaitAFull));
         if (!ok) break;
         ptx::tc_fence_after();
         const uint64_t bdesc = ptx::sw128_kmajor_desc(xs0 + sx * kXStageBytes);
@@ -203,7 +203,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     bool ok = true;
     for (int wb = wg; wb < WBs; wb += 2) {
       const int ws = wb % SW, sa = wb % SA;
-      ok = ptx::mbar_wait(full_w(ws), (wb / SW) & 1, err);
+      ok = ptx::mbar_wait(full_w(ws), (wb / SW) & 1, err, ptx::wait_code(ptx::kWaitGemm, ptx::kWaitWFull));
       if (!ok) break;
       // the row's 4 groups: 16*B bytes, read as 16-byte units
       uint32_t w[4 * B + 1];
@@ -217,7 +217,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       // the async-proxy refill of this stage must not overtake these reads
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(empty_w(ws));
-      ok = ptx::mbar_wait(empty_a(sa), ((wb / SA) & 1) ^ 1, err);
+      ok = ptx::mbar_wait(empty_a(sa), ((wb / SA) & 1) ^ 1, err, ptx::wait_code(ptx::kWaitGemm, ptx::kWaitAEmpty));
       if (!ok) break;
       ptx::tc_fence_after();
       const uint32_t col = tmem + lane_addr + kAccCols + sa * C::ACOLS;
@@ -235,7 +235,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       ptx::tc_fence_before();
       ptx::mbar_arrive(full_a(sa));
     }
-    if (ok) ok = ptx::mbar_wait(acc_full, 0, err);
+    if (ok) ok = ptx::mbar_wait(acc_full, 0, err, ptx::wait_code(ptx::kWaitGemm, ptx::kWaitAcc));
     if (ok) {
       ptx::tc_fence_after();
       const float sn = row_ok ? __ldg(scales + n) : 0.0f;

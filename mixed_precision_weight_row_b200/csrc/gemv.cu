@@ -463,11 +463,11 @@ cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* s
   // per-tile TMA kernel.  MPW_GEMV_KERNEL=mma selects the register-streaming
   // variant for canonical rows (tuning aid).
   static const bool use_mma = [] {
-    const char* e = getenv("MPW_GEMV_KERNEL");
+    const char* e = tuning_env("MPW_GEMV_KERNEL");
     return e != nullptr && e[0] == 'm';
   }();
   static const bool use_tc = [] {
-    const char* e = getenv("MPW_GEMV_KERNEL");
+    const char* e = tuning_env("MPW_GEMV_KERNEL");
     return e != nullptr && e[0] == 't' && e[1] == 'c';
   }();
   // Tensor-memory kernel (passes of 32 tokens) where it is the faster one

@@ -433,7 +433,7 @@ cudaError_t run_mma(const uint16_t* x, int M, const uint8_t* packed, const float
   Plan pl = plan_for(tiles, chunks, di.num_sms);
   // MPW_GEMV_CLUSTER=1|2|4|8 overrides the cluster size (tuning aid)
   static const int forced = [] {
-    const char* e = getenv("MPW_GEMV_CLUSTER");
+    const char* e = tuning_env("MPW_GEMV_CLUSTER");
     const int v = e ? atoi(e) : 0;
     return (v == 1 || v == 2 || v == 4 || v == 8) ? v : 0;
   }();

@@ -224,7 +224,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       int slot = 0;
       uint32_t phase = 0;
       for (; it.valid(); it.next()) {
-        if (!ptx::mbar_wait(empty(slot), phase, err)) break;
+        if (!ptx::mbar_wait(empty(slot), phase, err, ptx::wait_code(ptx::kWaitGemvSk, ptx::kWaitWEmpty))) break;
         issue_w(it, slot);
         issue_x(it, slot);
         ++issued;
@@ -234,7 +234,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         }
       }
       // nothing may still be landing in shared memory when the CTA exits
-      for (int s = max(0, issued - S); s < issued; ++s) ptx::mbar_wait(full(s % S), (s / S) & 1, err);
+      for (int s = max(0, issued - S); s < issued; ++s) ptx::mbar_wait(full(s % S), (s / S) & 1, err, ptx::wait_code(ptx::kWaitGemvSk, ptx::kWaitWTail));
     }
     return;
   }
@@ -350,7 +350,7 @@ gemv_sk_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   // walks every segment, so that all consumer warps meet at every barrier.
   bool ok = true;
   for (; it.valid(); it.next()) {
-    if (ok && !ptx::mbar_wait(full(slot), phase, err)) ok = false;
+    if (ok && !ptx::mbar_wait(full(slot), phase, err, ptx::wait_code(ptx::kWaitGemvSk, ptx::kWaitFull))) ok = false;
     const uint8_t* st = tsmem + st_off;
     const int nv = it.nv();
     if (ok) {
@@ -511,7 +511,7 @@ SkPlan plan_for(int M, int64_t N, int64_t K) {
   p.U = static_cast<int64_t>(p.T) * p.C;
   const int sms = device_info().num_sms;
   static const int cap = [] {
-    const char* e = getenv("MPW_GEMV_SK_CTAS");
+    const char* e = tuning_env("MPW_GEMV_SK_CTAS");
     const int v = e ? atoi(e) : 0;
     return v >= 1 && v <= 16 ? v : 0;
   }();

@@ -174,12 +174,12 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       int issued = 0;
       for (int i = 0; i < nkb; ++i) {
         const int s = i % SX;
-        if (!ptx::mbar_wait(empty_x(s), ((i / SX) & 1) ^ 1, err)) break;
+        if (!ptx::mbar_wait(empty_x(s), ((i / SX) & 1) ^ 1, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitXEmpty))) break;
         ptx::mbar_arrive_expect_tx(full_x(s), kXStageBytes);
         ptx::tma_load_2d(xs0 + s * kXStageBytes, &tmap_x, full_x(s), (kb0 + i) * BK, 0);
         issued = i + 1;
       }
-      for (int i = max(0, issued - SX); i < issued; ++i) ptx::mbar_wait(full_x(i % SX), (i / SX) & 1, err);
+      for (int i = max(0, issued - SX); i < issued; ++i) ptx::mbar_wait(full_x(i % SX), (i / SX) & 1, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitXTail));
     }
   } else if (warp == 3) {
     // ---------------- weight producer: one TMA per block ----------------
@@ -187,12 +187,12 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       int issued = 0;
       for (int i = 0; i < nwb; ++i) {
         const int s = i % SW;
-        if (!ptx::mbar_wait(empty_w(s), ((i / SW) & 1) ^ 1, err)) break;
+        if (!ptx::mbar_wait(empty_w(s), ((i / SW) & 1) ^ 1, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitWEmpty))) break;
         ptx::mbar_arrive_expect_tx(full_w(s), C::WSTAGE);
         ptx::tma_load_2d(ws0 + s * C::WSTAGE, &tmap_w, full_w(s), (wb0 + i) * 16 * B, n0);
         issued = i + 1;
       }
-      for (int i = max(0, issued - SW); i < issued; ++i) ptx::mbar_wait(full_w(i % SW), (i / SW) & 1, err);
+      for (int i = max(0, issued - SW); i < issued; ++i) ptx::mbar_wait(full_w(i % SW), (i / SW) & 1, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitWTail));
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -202,8 +202,8 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       for (int i = 0; i < nkb && ok; ++i) {
         const int sx = i % SX;
         const int wl = i >> 1, h = i & 1, sa = wl % SA;
-        ok = ptx::mbar_wait(full_x(sx), (i / SX) & 1, err);
-        if (ok && h == 0) ok = ptx::mbar_wait(full_a(sa), (wl / SA) & 1, err);
+        ok = ptx::mbar_wait(full_x(sx), (i / SX) & 1, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitFull));
+        if (ok && h == 0) ok = ptx::mbar_wait(full_a(sa), (wl / SA) & 1, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitAFull));
         if (!ok) break;
         ptx::tc_fence_after();
         const uint64_t bdesc = ptx::sw128_kmajor_desc(xs0 + sx * kXStageBytes);
@@ -235,7 +235,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       // the same in any order
       for (int i = 0; i < nkb; ++i) {
         const int s = i % SX;
-        if (!ptx::mbar_wait(full_x(s), (i / SX) & 1, err)) break;
+        if (!ptx::mbar_wait(full_x(s), (i / SX) & 1, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitSquares))) break;
         const uint4* row = reinterpret_cast<const uint4*>(smem + s * kXStageBytes + lane * 128);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -260,7 +260,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
     bool ok = true;
     for (int i = wg; i < nwb; i += C::NG) {
       const int ws = i % SW, sa = i % SA;
-      ok = ptx::mbar_wait(full_w(ws), (i / SW) & 1, err);
+      ok = ptx::mbar_wait(full_w(ws), (i / SW) & 1, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitWFull));
       if (!ok) break;
       uint32_t w[4 * B + 1];
       const uint8_t* stage = smem + SX * kXStageBytes + ws * C::WSTAGE;
@@ -272,7 +272,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       w[4 * B] = 0u;
       ptx::fence_proxy_async_smem();
       ptx::mbar_arrive(empty_w(ws));
-      ok = ptx::mbar_wait(empty_a(sa), ((i / SA) & 1) ^ 1, err);
+      ok = ptx::mbar_wait(empty_a(sa), ((i / SA) & 1) ^ 1, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitAEmpty));
       if (!ok) break;
       ptx::tc_fence_after();
       const uint32_t col = tmem + lane_addr + kAccCols + sa * C::ACOLS;
@@ -291,7 +291,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
       ptx::mbar_arrive(full_a(sa));
     }
     if (wg == 0) {
-      if (ok) ok = ptx::mbar_wait(acc_full, 0, err);
+      if (ok) ok = ptx::mbar_wait(acc_full, 0, err, ptx::wait_code(ptx::kWaitGemvTc, ptx::kWaitAcc));
 #pragma unroll
       for (int t = 0; t < BN; ++t) acc_row[t] = 0.0f;
       if (ok) {
@@ -367,7 +367,7 @@ gemv_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant
 template <int B>
 int tc_cluster(int tiles, int wbs, int M, int num_sms) {
   static const int forced = [] {
-    const char* e = getenv("MPW_GEMV_TC_CLUSTER");
+    const char* e = tuning_env("MPW_GEMV_TC_CLUSTER");
     const int v = e ? atoi(e) : 0;
     return v >= 1 && v <= kMaxCluster ? v : 0;
   }();

@@ -91,7 +91,7 @@ constexpr uint32_t kWholeSlice = 64u * 1024u;
 
 int ring_stages(int B, int M, int stages_per_cta, bool few_ctas, int ctas_by_regs, uint32_t fixed) {
   static const uint32_t budget = [] {
-    const char* e = getenv("MPW_GEMV_RING_KB");
+    const char* e = tuning_env("MPW_GEMV_RING_KB");
     const int v = e ? atoi(e) : 0;
     return v >= 8 && v <= 192 ? static_cast<uint32_t>(v) * 1024u : 0u;
   }();
@@ -255,7 +255,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
       int slot = 0;
       uint32_t phase = 0;   // phase of empty(slot) that frees it for stage s
       for (int s = pre; s < n_stages; ++s) {
-        if (!ptx::mbar_wait(empty(slot), phase, err)) break;
+        if (!ptx::mbar_wait(empty(slot), phase, err, ptx::wait_code(ptx::kWaitGemvTma, ptx::kWaitWEmpty))) break;
         issue_w(s, slot);
         issue_x(s, slot);
         issued = s + 1;
@@ -265,7 +265,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
         }
       }
       // nothing may still be landing in shared memory when the CTA exits
-      for (int s = max(0, issued - S); s < issued; ++s) ptx::mbar_wait(full(s % S), (s / S) & 1, err);
+      for (int s = max(0, issued - S); s < issued; ++s) ptx::mbar_wait(full(s % S), (s / S) & 1, err, ptx::wait_code(ptx::kWaitGemvTma, ptx::kWaitWTail));
     }
   } else {
     // ---------------- consumers ----------------
@@ -350,7 +350,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
     uint32_t phase = 0;
     uint32_t st_off = 0;
     for (int s = 0; s < n_stages; ++s) {
-      if (!ptx::mbar_wait(full(slot), phase, err)) break;
+      if (!ptx::mbar_wait(full(slot), phase, err, ptx::wait_code(ptx::kWaitGemvTma, ptx::kWaitFull))) break;
       const uint8_t* st = tsmem + st_off;
       const int c_first = cb + kSC * s + warp * kCH;
 #pragma unroll
@@ -494,7 +494,7 @@ int cluster_size(int tiles, int chunks, int num_sms) {
     }
   }
   static const int forced = [] {
-    const char* e = getenv("MPW_GEMV_CLUSTER");
+    const char* e = tuning_env("MPW_GEMV_CLUSTER");
     const int v = e ? atoi(e) : 0;
     return (v == 1 || v == 2 || v == 4 || v == 8) ? v : 0;
   }();

@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 namespace mpw {
 
@@ -20,6 +21,18 @@ constexpr int kLayoutPaired = 1;
 
 // Words (uint32) of one canonical packed row: 4 * ceil(K*b/128).
 inline int64_t row_words(int64_t K, int bits) { return 4 * ((K * bits + 127) / 128); }
+
+// Tuning aids for measurement: the MPW_GEMV_* environment variables are read
+// only in a library built with -DMPW_TUNING_KNOBS; the default build ignores
+// them, so the environment never changes which kernel runs or how.
+inline const char* tuning_env(const char* name) {
+#ifdef MPW_TUNING_KNOBS
+  return getenv(name);
+#else
+  (void)name;
+  return nullptr;
+#endif
+}
 
 // Per-device properties cached on first use.
 struct DeviceInfo {

@@ -64,18 +64,49 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
   return ok != 0;
 }
 
+// Codes a wait that gives up leaves in the device error word:
+// 100 * kernel + place.  The first one stays until the word is read.
+enum WaitKernel : int32_t { kWaitGemvTma = 1, kWaitGemvTc = 2, kWaitGemm = 3, kWaitGemvSk = 4 };
+enum WaitPlace : int32_t {
+  kWaitXEmpty = 1,    // x producer: a free x stage
+  kWaitXTail = 2,     // x producer: its last copies landed
+  kWaitWEmpty = 3,    // weight (or combined-stage) producer: a free stage
+  kWaitWTail = 4,     // weight (or combined-stage) producer: its last copies landed
+  kWaitFull = 5,      // consumer or MMA issuer: a loaded (x or combined) stage
+  kWaitAFull = 6,     // MMA issuer: converted weights in tensor memory
+  kWaitWFull = 7,     // converter: a loaded weight stage
+  kWaitAEmpty = 8,    // converter: a free tensor-memory stage
+  kWaitAcc = 9,       // epilogue: the finished accumulator
+  kWaitSquares = 10,  // sums of squares of x: a loaded x stage
+};
+__host__ __device__ constexpr int32_t wait_code(int32_t kernel, int32_t place) { return 100 * kernel + place; }
+
+// Timer steps longer than this between two reads of one waiting thread are
+// counted as this long, and backward steps as nothing: %globaltimer may be
+// adjusted while a kernel runs, and an adjustment must not end a wait early.
+constexpr uint64_t kWaitMaxStepNs = 1000000ull;
+// Backstop in polling rounds (each at least 128 try_waits, about a
+// microsecond or more), so that a wait also ends if the timer stands still.
+constexpr uint32_t kWaitMaxRounds = 1u << 23;
+
 // Waits for the phase with the given parity to complete.  Gives up after
-// `limit_ns` nanoseconds: sets *err to 1 and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* err,
+// `limit_ns` nanoseconds of waiting: stores `code` in *err unless an earlier
+// code is there, and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t* err, int32_t code,
                                           uint64_t limit_ns = 2000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
+  uint64_t prev = globaltimer();
+  uint64_t waited = 0;
+#pragma unroll 1
+  for (uint32_t round = 0;; ++round) {
 #pragma unroll 1
     for (int i = 0; i < 128; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > limit_ns) {
-      if (err != nullptr) atomicExch(err, 1);
+    const uint64_t now = globaltimer();
+    if (now > prev) waited += (now - prev < kWaitMaxStepNs) ? now - prev : kWaitMaxStepNs;
+    prev = now;
+    if (waited > limit_ns || round >= kWaitMaxRounds) {
+      if (err != nullptr) atomicCAS(err, 0, code);
       return false;
     }
   }

@@ -5,7 +5,9 @@ Every linear is checked against the oracle with the GPU's own bf16 input to
 that link (so errors do not compound along the chain): the oracle normalises
 that input itself where the link reads the rms-scaled input, quantizes a seeded sample of the
 matrix's rows and bounds the sampled outputs.  The whole pass issued as one
-mpw_recipe_run call must equal the link-by-link run bit for bit.
+mpw_recipe_run call must equal the link-by-link run bit for bit.  Both
+packed layouts are run at full size: the canonical rows and the paired
+halves the benchmark times.
 """
 import numpy as np
 import pytest
@@ -16,11 +18,15 @@ import workloads as wl
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def stack():
+@pytest.fixture(scope="module", params=["paired", "canonical"])
+def stack(request):
+    """The 448-matrix stack in the layout under test (paired: the layout the
+    benchmark times, re-ordered in place after quantization)."""
     import torch
 
     import mixed_precision_weight_row_b200 as mpw
+
+    layout = request.param
 
     shapes = wl.recipe_shapes()
     bits = wl.recipe_bits()
@@ -30,9 +36,13 @@ def stack():
         W = wl.gen_weight_torch(N, K, wl.RECIPE["sigma"], wl.recipe_weight_seed(i))
         packed, scales = mpw.quantize_pack(W, b)
         del W
-        layers.append(mpw.Linear(packed, scales, N, K, b, si, so, nrm))
+        if layout != "canonical":
+            mpw.repack(packed, K, b, "canonical", layout, out=packed)
+        layers.append(mpw.Linear(packed, scales, N, K, b, si, so, nrm, layout=layout))
     torch.cuda.synchronize()
-    return mpw, layers, shapes, bits
+    yield mpw, layers, shapes, bits
+    del layers
+    torch.cuda.empty_cache()
 
 
 def _slots(torch):

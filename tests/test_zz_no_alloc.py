@@ -6,6 +6,10 @@ ABI twice in a row and compares it with the existing entry point
 (mpw_qlinear_ex) and with the oracle, within the bound every decode test
 uses: |y - y_ref| <= 8e-3 * sum_k |x w_hat| + 1e-6.  Nothing here depends on
 what ran before, so the file passes alone or after the rest of the suite.
+
+Calls queued back to back on one stream, with no synchronisation between
+them, check that each call's clearing of the shared array lands after the
+previous call's kernel is done with it.
 """
 import numpy as np
 import pytest
@@ -87,3 +91,66 @@ def test_noalloc_rejects_what_its_scratch_cannot_hold(mpw):
                                        y.data_ptr(), 0) == mpw.MPW_E_INVALID_ARG
     assert mpw.lib.mpw_qlinear_noalloc(x.data_ptr() + 2, packed.data_ptr(), scales.data_ptr(), 6, 0, 1, 16, 64,
                                        y.data_ptr(), 0) == mpw.MPW_E_MISALIGNED
+
+
+@pytest.mark.parametrize("layout", ["paired", "canonical"])
+def test_noalloc_calls_queued_back_to_back(mpw, layout):
+    """Three calls on one stream (different x, separate outputs), one sync at
+    the end, on shapes with split tiles; M of 12 and 32 take the two- and
+    four-tile-wide kernels."""
+    import torch
+
+    rng = np.random.default_rng(4321)
+    for (N, K, b, M) in [(40, 17408, 5, 12), (40, 17408, 6, 32), (1024, 5120, 8, 32), (100, 2048, 11, 12)]:
+        W = rng.standard_normal((N, K)).astype(np.float32) * np.float32(0.02)
+        q, s = oracle.quantize(W, b)
+        packed = torch.from_numpy(oracle.pack_paired(q, b) if layout == "paired" else oracle.pack(q, b)).cuda()
+        scales = torch.from_numpy(s).cuda()
+        xs = [workloads.gen_x(M, K, seed=77 * N + call).cuda() for call in range(3)]
+        ys = [torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+        ye = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+        for x, y in zip(xs, ys):
+            assert _call_noalloc(mpw, x, packed, scales, b, layout, y) == mpw.MPW_OK
+        for x, y in zip(xs, ye):
+            assert _call_existing(mpw, x, packed, scales, b, layout, y) == mpw.MPW_OK
+        torch.cuda.synchronize()
+        for x, y, e in zip(xs, ys, ye):
+            y_ref, bound = oracle.qlinear_ref(x.float().cpu().numpy(), q, s)
+            a = y.float().cpu().numpy()
+            assert oracle.check_qlinear(a, y_ref, bound).all(), (N, K, b, M)
+            assert (np.abs(a - e.float().cpu().numpy()) <= 2 * bound).all()
+    assert mpw.device_error() == 0
+
+
+def test_noalloc_limit_agrees_with_workspace_size(mpw):
+    """On the 27B-class MLP shapes, the call is refused exactly when the
+    workspace it needs (mpw_qlinear_workspace_bytes) exceeds the array.  The
+    buffers have their full sizes (zero weights, zero x), so a call that does
+    run reads only what it owns and writes zeros."""
+    import torch
+
+    limit = 4 << 20
+    refused = 0
+    for (N, K) in [(17408, 5120), (5120, 17408)]:
+        for b in (5, 6):
+            rb = mpw.packed_row_bytes(K, b)
+            packed = torch.zeros((N, rb), dtype=torch.uint8, device="cuda")
+            scales = torch.ones(N, dtype=torch.float32, device="cuda")
+            for M in (1, 8, 32):
+                need = mpw.lib.mpw_qlinear_workspace_bytes(b, mpw.LAYOUTS["paired"], M, N, K)
+                x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+                y = torch.full((M, N), 7.0, dtype=torch.bfloat16, device="cuda")
+                if N == 17408:
+                    # what the header states for the gate/up shape
+                    assert (need > limit) == (M == 32), (b, M, need)
+                st = _call_noalloc(mpw, x, packed, scales, b, "paired", y)
+                if need > limit:
+                    refused += 1
+                    assert st == mpw.MPW_E_SCRATCH_LIMIT, (N, K, b, M, need)
+                else:
+                    assert st == mpw.MPW_OK, (N, K, b, M, need)
+                    torch.cuda.synchronize()
+                    assert float(y.float().abs().max()) == 0.0
+    # gate/up at M = 32 needs more than the array holds
+    assert refused >= 1
+    assert mpw.device_error() == 0
