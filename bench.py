@@ -365,6 +365,54 @@ def measure_quantize(mpw, W_gpu, b, steps, warmup, l2_bytes):
             "weights_per_s": N * K / (per * 1e-6), "copies": copies}
 
 
+def measure_groups(mpw, W_gpu, b, g, l2_bytes, layout, steps, warmup=3):
+    """Group-wise scales (one per g weights of a row): the quantizer, and the
+    decode GEMV at M = 1 over a pool of distinct copies, flagged like the
+    headline (x_ready + y_unshared).  GB/s count the packed codes and the
+    group scales."""
+    import torch
+
+    import workloads as wl
+
+    N, K = W_gpu.shape
+    packed, scales = mpw.quantize_pack_groups(W_gpu, b, g)
+    torch.cuda.synchronize()
+    # quantizer: distinct W copies > 4x L2
+    copies = max(2, -(-4 * l2_bytes // (N * K * 4)))
+    Ws = [W_gpu.clone() for _ in range(copies)]
+
+    def qstep():
+        for Wc in Ws:
+            mpw.quantize_pack_groups(Wc, b, g, packed=packed, scales=scales)
+
+    gq = graph_of(qstep)
+    qms = time_graph(gq, 20, warmup)
+    del gq, Ws
+    q_us = qms * 1e3 / (20 * copies)
+    q_bytes = N * K * 4 + packed.numel() + scales.numel() * 4
+    if layout != "canonical":
+        packed = mpw.repack(packed, K, b, "canonical", layout)
+    per = packed.numel() + scales.numel() * 4
+    P = max(2, -(-4 * l2_bytes // per))
+    pk = [packed.clone() for _ in range(P)]
+    sc = [scales.clone() for _ in range(P)]
+    x = wl.gen_x(1, K, wl.DECODE["x_seed"]).cuda()
+    ys = torch.empty((P, 1, N), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        for i in range(P):
+            mpw.qlinear_groups(x, pk[i], sc[i], b, g, y=ys[i], layout=layout, x_ready=True, y_unshared=True)
+
+    gd = graph_of(step)
+    ms = time_graph(gd, steps, warmup)
+    del gd
+    us = ms * 1e3 / (steps * P)
+    return {"b": b, "group": g, "layout": layout, "scale_bytes": scales.numel() * 4,
+            "us_per_launch": round(us, 4), "weight_GBps": round(per / (us * 1e3), 1),
+            "alg_GBps": round((per + 2 * K + 2 * N) / (us * 1e3), 1),
+            "quantize_us": round(q_us, 3), "quantize_GBps": round(q_bytes / (q_us * 1e3), 1)}
+
+
 def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup, pool_n, layout="canonical",
                 world=1):
     """Same metric through the public call with host buffers: each step copies
@@ -761,6 +809,15 @@ def main(argv=None):
                 r["pct_hbm"] = 100.0 * r["alg_GBps"] / pk["hbm_gbs"]
                 extras["quantize_pack"].append({k: (round(v, 4) if isinstance(v, float) else v)
                                                 for k, v in r.items()})
+        groups = []
+        for b in (4, 6):
+            for gsize in (128, 256):
+                r = sec.run(f"groups b={b} g={gsize}", measure_groups, mpw, W, b, gsize, l2, lay,
+                            max(20, args.steps // 4))
+                if r is not None:
+                    r["pct_hbm"] = round(100.0 * r["alg_GBps"] / pk["hbm_gbs"], 2)
+                    groups.append(r)
+        extras["group_scales"] = groups
         mlp = []
         for name, n_, k_ in wl.MLP27B["shapes"][1:]:
             Wm = wl.gen_weight_torch(n_, k_, wl.MLP27B["sigma"], 17 + n_)

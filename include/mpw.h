@@ -184,6 +184,42 @@ MPW_API mpw_status mpw_qlinear_ex(const uint16_t* x, const uint8_t* packed, cons
                                   uint16_t* y, int path, mpw_stream_t stream);
 
 /*
+ * Group-wise scales (quantization tutorial, exercises, item 1: one scale per
+ * 128 weights instead of one per output channel; group sizes 32, 64, 128 and
+ * 256 compared).  Groups are `group` consecutive weights of a row along K,
+ * the last one shorter when group does not divide K; each group is quantized
+ * with the per-row formula above applied to the group (s_nj = fl32(max |w| /
+ * Q) over group j, a zero group takes fl32(1 / Q)).  The codes are stored in
+ * the canonical packed format (mpw_unpack reads them; mpw_repack re-orders
+ * them), the scales as fp32 [N, ceil(K / group)] row-major.
+ *
+ * mpw_quantize_pack_groups -- group-wise quantization and canonical packing.
+ *   group    a power of two in 32..1024 (else MPW_E_INVALID_ARG).
+ *   W, packed, nonfinite_flag  as for mpw_quantize_pack.
+ *   scales   device, fp32 [N, ceil(K / group)].
+ */
+MPW_API mpw_status mpw_quantize_pack_groups(const float* W, int64_t N, int64_t K, int bits, int64_t group,
+                                            uint8_t* packed, float* scales, int32_t* nonfinite_flag,
+                                            mpw_stream_t stream);
+
+/*
+ * mpw_qlinear_groups -- y = x @ (q * s_group)^T for group-scaled rows:
+ *   y[m, n] = bf16_rn(sum_j s_nj * sum_{k in group j} x[m, k] q[n, k]), each
+ *   group's sum in fp32, scaled in fp32 and added to an fp32 accumulator.
+ *   group    a power of two in 128..1024 (a group then holds whole 128-code
+ *            chunks of the decode kernel); smaller groups: MPW_E_INVALID_ARG.
+ *   layout   MPW_LAYOUT_* of `packed`.
+ *   M >= 1, run as the decode kernel in passes of 32 tokens; K % 8 == 0
+ *   (K % 32 == 0 for paired rows); x 16-byte aligned (else MPW_E_MISALIGNED).
+ *   flags    0, MPW_QLINEAR_X_READY or MPW_QLINEAR_X_READY |
+ *            MPW_QLINEAR_Y_UNSHARED, with the meaning they have for
+ *            mpw_qlinear_flags (defined below).
+ */
+MPW_API mpw_status mpw_qlinear_groups(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                                      int64_t group, int layout, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                      unsigned flags, mpw_stream_t stream);
+
+/*
  * Workspace of the decode kernels.  For M <= 32 the fastest decode kernel
  * splits the (16-row tile, 128-code chunk) units of W evenly over a
  * persistent grid; a tile shared by two or more CTAs is combined through a
@@ -426,6 +462,21 @@ MPW_API mpw_status mpw_file_read(const char* path, int64_t index, uint8_t* packe
 MPW_API mpw_status mpw_qlinear_noalloc(const uint16_t* x, const uint8_t* packed, const float* scales,
                                        int bits, int layout, int64_t M, int64_t N, int64_t K,
                                        uint16_t* y, mpw_stream_t stream);
+
+/*
+ * mpw_gather_shards -- re-orders the gathered outputs of an output-row
+ * (N) sharded linear into y.  No page describes tensor parallelism; the
+ * partition is this library's: rank r of `world` owns weight rows
+ * r * Nl .. r * Nl + Nl - 1 (zero rows past N) and computes y_r [M, Nl] for
+ * the replicated x; an all-gather of the y_r (NCCL, by the caller) leaves
+ * blocks [world, M, Nl] rank after rank.
+ *   blocks  device, bf16 [world, M, Nl].
+ *   y       device, bf16 [M, N]: y[m, n] = blocks[n / Nl, m, n % Nl].
+ *   N <= world * Nl.  For M = 1 the blocks already are y (the first N
+ *   values) and no call is needed.
+ */
+MPW_API mpw_status mpw_gather_shards(const uint16_t* blocks, int64_t world, int64_t M, int64_t Nl, int64_t N,
+                                     uint16_t* y, mpw_stream_t stream);
 
 /*
  * mpw_device_error -- synchronises the current device, returns in *code the

@@ -19,7 +19,8 @@ __all__ = [
     "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
     "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str", "allocate_bits", "allocation_frontier",
     "recipe_plan", "save_packed", "load_packed",
-    "LAYOUTS", "workspace", "qlinear_workspace_bytes",
+    "LAYOUTS", "workspace", "qlinear_workspace_bytes", "quantize_pack_groups", "qlinear_groups",
+    "gather_shards",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmpw.so")
@@ -135,6 +136,12 @@ def _load():
     L.mpw_qlinear_noalloc.restype = c_int
     L.mpw_recipe_run.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp]
     L.mpw_recipe_run.restype = c_int
+    L.mpw_quantize_pack_groups.argtypes = [vp, i64, i64, c_int, i64, vp, vp, vp, vp]
+    L.mpw_quantize_pack_groups.restype = c_int
+    L.mpw_qlinear_groups.argtypes = [vp, vp, vp, c_int, i64, c_int, i64, i64, i64, vp, ctypes.c_uint, vp]
+    L.mpw_qlinear_groups.restype = c_int
+    L.mpw_gather_shards.argtypes = [vp, i64, i64, i64, i64, vp, vp]
+    L.mpw_gather_shards.restype = c_int
     L.mpw_device_error.argtypes = [ctypes.POINTER(i32)]
     L.mpw_device_error.restype = c_int
     return L
@@ -333,6 +340,72 @@ def qlinear(x, packed, scales, bits: int, y=None, path: str = "auto", layout: st
     _check(lib.mpw_qlinear_ws(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits), LAYOUTS[layout],
                               M, N, K, y.data_ptr(), PATHS[path], None if ws is None else ws.data_ptr(),
                               ws_bytes, _stream(stream)), "mpw_qlinear")
+    return y
+
+
+def quantize_pack_groups(W, bits: int, group: int, packed=None, scales=None, nonfinite_flag=None, stream=None):
+    """W fp32 [N, K] (CUDA) -> (packed uint8 [N, row_bytes], scales fp32
+    [N, ceil(K / group)]): one scale per ``group`` consecutive weights of a
+    row (mpw_quantize_pack_groups)."""
+    import torch
+
+    _need(W, torch.float32, "W", 2)
+    N, K = W.shape
+    rb = packed_row_bytes(K, bits)
+    G = -(-K // int(group)) if group > 0 else 0
+    if packed is None:
+        packed = torch.empty((N, max(rb, 16)), dtype=torch.uint8, device=W.device)
+    if scales is None:
+        scales = torch.empty((N, max(G, 1)), dtype=torch.float32, device=W.device)
+    _need(packed, torch.uint8, "packed")
+    _need(scales, torch.float32, "scales")
+    flag = 0 if nonfinite_flag is None else nonfinite_flag.data_ptr()
+    _check(lib.mpw_quantize_pack_groups(W.data_ptr(), N, K, int(bits), int(group), packed.data_ptr(),
+                                        scales.data_ptr(), flag, _stream(stream)), "mpw_quantize_pack_groups")
+    return packed, scales
+
+
+def qlinear_groups(x, packed, scales, bits: int, group: int, y=None, layout: str = "canonical", stream=None,
+                   x_ready: bool = False, y_unshared: bool = False):
+    """y = x @ (q * s_group)^T with group scales [N, ceil(K / group)]
+    (mpw_qlinear_groups); x bf16 [M, K] -> y bf16 [M, N].  ``x_ready`` and
+    ``y_unshared`` as for qlinear."""
+    import torch
+
+    _need(x, torch.bfloat16, "x", 2)
+    _need(packed, torch.uint8, "packed", 2)
+    _need(scales, torch.float32, "scales", 2)
+    M, K = x.shape
+    N = packed.shape[0]
+    if scales.shape[0] != N or scales.shape[1] != -(-K // int(group)):
+        raise ValueError("scales must be [N, ceil(K / group)]")
+    if packed.shape[1] != packed_row_bytes(K, bits):
+        raise ValueError("packed rows must be exactly packed_row_bytes(K, bits) long")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(y, torch.bfloat16, "y")
+    if y_unshared and not x_ready:
+        raise ValueError("y_unshared needs x_ready")
+    flags = (X_READY if x_ready else 0) | (Y_UNSHARED if y_unshared else 0)
+    _check(lib.mpw_qlinear_groups(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits), int(group),
+                                  LAYOUTS[layout], M, N, K, y.data_ptr(), flags, _stream(stream)),
+           "mpw_qlinear_groups")
+    return y
+
+
+def gather_shards(blocks, world: int, M: int, Nl: int, N: int, y=None, stream=None):
+    """Gathered outputs of an N-sharded linear, bf16 [world * M * Nl] rank
+    after rank, -> y bf16 [M, N] (mpw_gather_shards; see shard.py)."""
+    import torch
+
+    _need(blocks, torch.bfloat16, "blocks")
+    if blocks.numel() != world * M * Nl:
+        raise ValueError("blocks must hold world * M * Nl values")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=blocks.device)
+    _need(y, torch.bfloat16, "y", 2)
+    _check(lib.mpw_gather_shards(blocks.data_ptr(), int(world), int(M), int(Nl), int(N), y.data_ptr(),
+                                 _stream(stream)), "mpw_gather_shards")
     return y
 
 

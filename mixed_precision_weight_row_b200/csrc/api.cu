@@ -186,6 +186,46 @@ mpw_status mpw_repack(const uint8_t* in, int64_t N, int64_t K, int bits, int lay
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+mpw_status mpw_quantize_pack_groups(const float* W, int64_t N, int64_t K, int bits, int64_t group, uint8_t* packed,
+                                    float* scales, int32_t* nonfinite_flag, mpw_stream_t stream) {
+  if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
+  if (W == nullptr || packed == nullptr || scales == nullptr || N < 1 || K < 1) return MPW_E_INVALID_ARG;
+  if (group < 32 || group > 1024 || (group & (group - 1)) != 0) return MPW_E_INVALID_ARG;
+  if (N > 0x7fffffff || K > 0x3fffffff) return MPW_E_INVALID_ARG;
+  // one warp per 1024 weights of a row: the grid must stay below 2^31 blocks
+  if (N * (((K + 31) / 32 + 31) / 32) > (int64_t{1} << 36)) return MPW_E_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(W, 4) || !aligned(scales, 4) ||
+      (nonfinite_flag != nullptr && !aligned(nonfinite_flag, 4)))
+    return MPW_E_MISALIGNED;
+  return from_cuda(launch_quantize_pack_groups(W, N, K, bits, group, packed, scales, nonfinite_flag,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mpw_status mpw_qlinear_groups(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int64_t group,
+                              int layout, int64_t M, int64_t N, int64_t K, uint16_t* y, unsigned flags,
+                              mpw_stream_t stream) {
+  if (!bits_ok(bits)) return MPW_E_UNSUPPORTED_BITS;
+  if ((flags & ~static_cast<unsigned>(MPW_QLINEAR_X_READY | MPW_QLINEAR_Y_UNSHARED)) != 0) return MPW_E_INVALID_ARG;
+  if ((flags & MPW_QLINEAR_Y_UNSHARED) && !(flags & MPW_QLINEAR_X_READY)) return MPW_E_INVALID_ARG;
+  if (x == nullptr || packed == nullptr || scales == nullptr || y == nullptr || M < 1 || N < 1 || K < 1)
+    return MPW_E_INVALID_ARG;
+  if (N > 0x7fffffff || K > 0x3fffffff || M > 0x7fffffff || !layout_ok(layout)) return MPW_E_INVALID_ARG;
+  if (group < 128 || group > 1024 || (group & (group - 1)) != 0) return MPW_E_INVALID_ARG;
+  if (K % 8 != 0 || (layout == MPW_LAYOUT_PAIRED && K % 32 != 0)) return MPW_E_INVALID_ARG;
+  if (!aligned(packed, 16) || !aligned(x, 16) || !aligned(y, 2) || !aligned(scales, 4)) return MPW_E_MISALIGNED;
+  if (!gemv_groups_supported(x, M, N, K, group)) return MPW_E_CUDA;   // no tensor-map encoder
+  return from_cuda(launch_gemv_groups(x, packed, scales, bits, group, layout, M, N, K, y,
+                                      reinterpret_cast<cudaStream_t>(stream), flags));
+}
+
+mpw_status mpw_gather_shards(const uint16_t* blocks, int64_t world, int64_t M, int64_t Nl, int64_t N, uint16_t* y,
+                             mpw_stream_t stream) {
+  if (blocks == nullptr || y == nullptr || world < 1 || M < 1 || Nl < 1 || N < 1) return MPW_E_INVALID_ARG;
+  if (world > 0x10000 || M > 0x7fffffff || Nl > 0x7fffffff || N > world * Nl) return MPW_E_INVALID_ARG;
+  if (!aligned(blocks, 2) || !aligned(y, 2)) return MPW_E_MISALIGNED;
+  return from_cuda(launch_gather_shards(blocks, M, Nl, N, y, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 namespace {
 
 mpw_status qlinear_impl(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,

@@ -58,6 +58,10 @@ cudaError_t ensure_smem_attr(const void* kernel, size_t bytes);
 cudaError_t launch_quantize_pack(const float* W, int64_t N, int64_t K, int bits,
                                  uint8_t* packed, float* scales, int32_t* flag,
                                  cudaStream_t stream);
+// Group-wise scales: one per `group` consecutive weights of a row (a power of
+// two in 32..1024); scales [N, ceil(K / group)].
+cudaError_t launch_quantize_pack_groups(const float* W, int64_t N, int64_t K, int bits, int64_t group,
+                                        uint8_t* packed, float* scales, int32_t* flag, cudaStream_t stream);
 cudaError_t launch_unpack(const uint8_t* packed, int64_t N, int64_t K, int bits,
                           int16_t* codes, cudaStream_t stream);
 cudaError_t launch_dequantize(const uint8_t* packed, const float* scales, int64_t N,
@@ -123,6 +127,18 @@ bool gemv_tc_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, bool 
 bool gemv_tc_preferred(int bits, int64_t M, int64_t N, int64_t K);
 cudaError_t launch_gemv_tc(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,
                            int64_t M, int64_t N, int64_t K, uint16_t* y, bool norm, cudaStream_t stream);
+
+// gemv_group.cu: decode linear with group-wise scales (group a power of two
+// in 128..1024; scales [N, ceil(K / group)]) on the per-tile TMA kernel, in
+// passes of 32 tokens.
+bool gemv_groups_supported(const uint16_t* x, int64_t M, int64_t N, int64_t K, int64_t group);
+cudaError_t launch_gemv_groups(const uint16_t* x, const uint8_t* packed, const float* scales, int bits,
+                               int64_t group, int layout, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                               cudaStream_t stream, unsigned qflags = 0u);
+
+// shard.cu: gathered output blocks [world, M, Nl] -> y [M, N] (N <= world * Nl).
+cudaError_t launch_gather_shards(const uint16_t* blocks, int64_t M, int64_t Nl, int64_t N, uint16_t* y,
+                                 cudaStream_t stream);
 
 // gemm.cu: tcgen05 prefill GEMM; returns cudaErrorNotSupported for shapes it
 // does not take (the caller then uses the GEMV path).

@@ -163,6 +163,70 @@ quantize_pack_kernel(const float* __restrict__ W, int K, int rw, uint8_t* __rest
 }
 
 // ---------------------------------------------------------------------------
+// group-wise scales: one scale per g consecutive weights of a row
+// ---------------------------------------------------------------------------
+
+// Quantization tutorial, exercises, item 1 (one scale per 128 weights; 32,
+// 64, 128 and 256 compared), with the per-channel formula of "How
+// quantization works" applied to each group.  One warp covers 1024
+// consecutive weights of a row: lane l quantizes the 32-code unit l (its 32
+// weights in registers) into exactly B words.  A group is 1 << gu_log2 units
+// (g = 32 .. 1024, a power of two), so groups never straddle warps and a
+// group's maximum is a butterfly over its lanes.  Units past K hold zeros.
+template <int B>
+__global__ void __launch_bounds__(256)
+quantize_pack_groups_kernel(const float* __restrict__ W, int64_t N, int K, int rw, int gu_log2, int G,
+                            uint8_t* __restrict__ packed, float* __restrict__ scales,
+                            int32_t* __restrict__ flag, bool vec4) {
+  const int lane = threadIdx.x & 31;
+  const int U = (K + 31) >> 5;           // 32-code units per row
+  const int wpr = (U + 31) >> 5;         // warps per row
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) >> 5;
+  if (wid >= N * wpr) return;            // the whole warp leaves together
+  const int64_t n = wid / wpr;
+  const int wr = static_cast<int>(wid - n * wpr);
+  const int u = wr * 32 + lane;
+  const int k0 = u * 32;
+  const float* row = W + n * K;
+  float v[32];
+  if (vec4 && k0 + 32 <= K) {
+    const float4* r4 = reinterpret_cast<const float4*>(row + k0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 t = __ldg(r4 + i);
+      v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = (k0 + j < K) ? __ldg(row + k0 + j) : 0.0f;
+  }
+  float m = 0.0f;
+  bool bad = false;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    m = fmaxf(m, fabsf(v[j]));
+    bad |= !isfinite(v[j]);
+  }
+  if (bad && flag != nullptr) *flag = 1;
+  for (int o = 1; o < (1 << gu_log2); o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float s = row_scale<B>(m);
+  if (u < U && (lane & ((1 << gu_log2) - 1)) == 0) scales[n * G + (u >> gu_log2)] = s;
+  uint32_t w[B];
+  pack_group<B>(s, [&](int j) { return v[j]; }, w);
+  uint32_t* out = reinterpret_cast<uint32_t*>(packed + static_cast<size_t>(n) * rw * 4);
+  if (u < U) {
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+      const int idx = u * B + i;
+      if (idx < rw) out[idx] = w[i];
+    }
+  }
+  // zero the words past the last unit (padding up to the 16-byte row stride)
+  if (wr == wpr - 1)
+    for (int idx = U * B + lane; idx < rw; idx += 32) out[idx] = 0u;
+}
+
+// ---------------------------------------------------------------------------
 // unpack / dequantize: one thread per group of 32 codes
 // ---------------------------------------------------------------------------
 
@@ -252,6 +316,23 @@ struct QuantizeLaunch {
   }
 };
 
+template <int B>
+struct QuantizeGroupsLaunch {
+  static cudaError_t run(const float* W, int64_t N, int64_t K, int64_t group, uint8_t* packed, float* scales,
+                         int32_t* flag, cudaStream_t stream) {
+    const int rw = static_cast<int>(row_words(K, B));
+    int gl = 0;
+    while ((int64_t{32} << gl) < group) ++gl;
+    const int G = static_cast<int>((K + group - 1) / group);
+    const int64_t wpr = ((K + 31) / 32 + 31) / 32;
+    const int64_t blocks = (N * wpr * 32 + 255) / 256;
+    const bool vec4 = (K % 4 == 0) && (reinterpret_cast<uintptr_t>(W) % 16 == 0);
+    quantize_pack_groups_kernel<B><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        W, N, static_cast<int>(K), rw, gl, G, packed, scales, flag, vec4);
+    return cudaGetLastError();
+  }
+};
+
 unsigned grid_for(int64_t work, int threads) {
   const int64_t blocks = (work + threads - 1) / threads;
   const int64_t cap = static_cast<int64_t>(device_info().num_sms) * 16;
@@ -279,6 +360,11 @@ struct UnpackLaunch {
 cudaError_t launch_quantize_pack(const float* W, int64_t N, int64_t K, int bits, uint8_t* packed,
                                  float* scales, int32_t* flag, cudaStream_t stream) {
   return dispatch_bits<QuantizeLaunch>(bits, W, N, K, packed, scales, flag, stream);
+}
+
+cudaError_t launch_quantize_pack_groups(const float* W, int64_t N, int64_t K, int bits, int64_t group,
+                                        uint8_t* packed, float* scales, int32_t* flag, cudaStream_t stream) {
+  return dispatch_bits<QuantizeGroupsLaunch>(bits, W, N, K, group, packed, scales, flag, stream);
 }
 
 cudaError_t launch_unpack(const uint8_t* packed, int64_t N, int64_t K, int bits, int16_t* codes,

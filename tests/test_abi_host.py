@@ -233,3 +233,30 @@ def test_product_path_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".h", ".cuh")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_group_entry_points_validation():
+    """Group-wise scales: the group size, shapes, layout and alignment are
+    checked before anything is launched."""
+    L = mpw.lib
+    qg = L.mpw_quantize_pack_groups
+    assert qg(A16, 4, 256, 3, 128, A16B, A16, 0, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    for bad_group in (0, 16, 48, 96, 2048, -128):
+        assert qg(A16, 4, 256, 5, bad_group, A16B, A16, 0, 0) == mpw.MPW_E_INVALID_ARG, bad_group
+    assert qg(0, 4, 256, 5, 128, A16B, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert qg(A16, 0, 256, 5, 128, A16B, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert qg(A16, 4, 256, 5, 128, A16B + 8, A16, 0, 0) == mpw.MPW_E_MISALIGNED
+    assert qg(A16, 4, 256, 5, 128, A16B, A16 + 2, 0, 0) == mpw.MPW_E_MISALIGNED
+    ql = L.mpw_qlinear_groups
+    # x, packed, scales, bits, group, layout, M, N, K, y, stream
+    assert ql(A16, A16B, A16, 16, 128, 0, 1, 16, 256, A16, 0, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    for bad_group in (32, 64, 100, 2048):
+        assert ql(A16, A16B, A16, 5, bad_group, 0, 1, 16, 256, A16, 0, 0) == mpw.MPW_E_INVALID_ARG, bad_group
+    assert ql(A16, A16B, A16, 5, 128, 2, 1, 16, 256, A16, 0, 0) == mpw.MPW_E_INVALID_ARG      # layout
+    assert ql(A16, A16B, A16, 5, 128, 0, 0, 16, 256, A16, 0, 0) == mpw.MPW_E_INVALID_ARG      # M
+    assert ql(A16, A16B, A16, 5, 128, 0, 1, 16, 250, A16, 0, 0) == mpw.MPW_E_INVALID_ARG      # K % 8
+    assert ql(A16, A16B, A16, 5, 128, 1, 1, 16, 264, A16, 0, 0) == mpw.MPW_E_INVALID_ARG      # paired K % 32
+    assert ql(A16 + 8, A16B, A16, 5, 128, 0, 1, 16, 256, A16, 0, 0) == mpw.MPW_E_MISALIGNED  # x 16-byte
+    assert ql(0, A16B, A16, 5, 128, 0, 1, 16, 256, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
+    assert ql(A16, A16B, A16, 5, 128, 0, 1, 16, 256, A16, 2, 0) == mpw.MPW_E_INVALID_ARG   # y_unshared alone
+    assert ql(A16, A16B, A16, 5, 128, 0, 1, 16, 256, A16, 4, 0) == mpw.MPW_E_INVALID_ARG   # unknown flag
