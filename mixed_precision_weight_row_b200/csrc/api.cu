@@ -192,8 +192,8 @@ mpw_status mpw_quantize_pack_groups(const float* W, int64_t N, int64_t K, int bi
   if (W == nullptr || packed == nullptr || scales == nullptr || N < 1 || K < 1) return MPW_E_INVALID_ARG;
   if (group < 32 || group > 1024 || (group & (group - 1)) != 0) return MPW_E_INVALID_ARG;
   if (N > 0x7fffffff || K > 0x3fffffff) return MPW_E_INVALID_ARG;
-  // one warp per 1024 weights of a row: the grid must stay below 2^31 blocks
-  if (N * (((K + 31) / 32 + 31) / 32) > (int64_t{1} << 36)) return MPW_E_INVALID_ARG;
+  // one warp per 1024 weights of a row, 8 warps per block: under 2^31 blocks
+  if (N * (((K + 31) / 32 + 31) / 32) >= (int64_t{1} << 34)) return MPW_E_INVALID_ARG;
   if (!aligned(packed, 16) || !aligned(W, 4) || !aligned(scales, 4) ||
       (nonfinite_flag != nullptr && !aligned(nonfinite_flag, 4)))
     return MPW_E_MISALIGNED;
