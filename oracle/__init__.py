@@ -34,3 +34,11 @@ from .quant import (  # noqa: F401
     unpack_paired,
     unpadded_row_bytes,
 )
+from .fp8 import (  # noqa: F401
+    E4M3_MAX,
+    FP8_MAX_BITS,
+    e4m3_round,
+    fp8_input_error_bound,
+    qlinear_fp8_ref,
+    quantize_x_fp8,
+)
