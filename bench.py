@@ -197,7 +197,8 @@ class Pool:
 
 
 # Where a code in the device error word comes from: 100 * kernel + place.
-WAIT_KERNELS = {1: "gemv_tma_kernel", 2: "gemv_tc_kernel", 3: "gemm_kernel", 4: "gemv_sk_kernel"}
+WAIT_KERNELS = {1: "gemv_tma_kernel", 2: "gemv_tc_kernel", 3: "gemm_kernel", 4: "gemv_sk_kernel",
+                5: "gemm_fp8_kernel"}
 WAIT_PLACES = {1: "x producer: free x stage", 2: "x producer: last copies", 3: "producer: free stage",
                4: "producer: last copies", 5: "consumer / MMA issuer: loaded stage",
                6: "MMA issuer: converted weights", 7: "converter: loaded weight stage",
@@ -488,6 +489,56 @@ def measure_prefill(mpw, pk, reps=10, layout="canonical"):
             out.append({"shape": f"{name} {N}x{K}", "b": b, "us": round(us, 2), "TFLOPs": round(tf, 1),
                         "pct_bf16_peak": round(100 * tf / pk["bf16_tflops"], 2),
                         "executed_mma_TFLOPs": round(executed, 1)})
+            del packed, scales, y
+        del W
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_prefill_fp8(mpw, pk, reps=10, layout="canonical"):
+    """FP8 (E4M3) prefill GEMM for 4- and 5-bit codes on the prefill shapes:
+    x 2048x5120 quantized per token once (timed apart), then the GEMM.
+    The FP8 tensor-core peak is taken as twice the measured bf16 one (the
+    nominal ratio of the two dense rates)."""
+    import torch
+
+    import workloads as wl
+
+    c = wl.PREFILL
+    x = wl.gen_x(c["M"], 5120, c["x_seed"]).cuda()
+    xq, sx = mpw.quantize_x_fp8(x)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        mpw.quantize_x_fp8(x, xq=xq, sx=sx)
+    e1.record()
+    torch.cuda.synchronize()
+    xq_us = e0.elapsed_time(e1) * 1e3 / reps
+    fp8_peak = 2.0 * pk["bf16_tflops"]
+    out = []
+    for name, N, K in c["shapes"]:
+        W = wl.gen_weight_torch(N, K, c["sigma"], 11 + N)
+        for b in (4, 5):
+            packed, scales = mpw.quantize_pack(W, b)
+            if layout != "canonical":
+                packed = mpw.repack(packed, K, b, "canonical", layout)
+            y = torch.empty((c["M"], N), dtype=torch.bfloat16, device="cuda")
+            for _ in range(3):
+                mpw.qlinear_fp8(x, packed, scales, b, y=y, layout=layout, xq=xq, sx=sx)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(reps):
+                mpw.qlinear_fp8(x, packed, scales, b, y=y, layout=layout, xq=xq, sx=sx)
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / reps
+            tf = 2.0 * c["M"] * N * K / (us * 1e-6) / 1e12
+            out.append({"shape": f"{name} {N}x{K}", "b": b, "us": round(us, 2), "TFLOPs": round(tf, 1),
+                        "pct_fp8_peak": round(100 * tf / fp8_peak, 2),
+                        "pct_bf16_peak": round(100 * tf / pk["bf16_tflops"], 2),
+                        "x_quantize_us": round(xq_us, 2)})
             del packed, scales, y
         del W
         torch.cuda.empty_cache()
@@ -839,11 +890,14 @@ def main(argv=None):
             torch.cuda.empty_cache()
         extras["mlp27b"] = mlp
         extras["prefill"] = sec.run("prefill", measure_prefill, mpw, pk, layout=lay)
+        extras["prefill_fp8"] = sec.run("prefill_fp8", measure_prefill_fp8, mpw, pk, layout=lay)
         extras["allocator"] = sec.run("allocator", measure_allocator, mpw)
         extras["recipe"] = sec.run("recipe", measure_recipe, mpw, pk, layout=lay)
         summary = {}
         for p in extras.get("prefill") or []:
             summary[f"prefill {p['shape']} b={p['b']} TFLOPs"] = p["TFLOPs"]
+        for p in extras.get("prefill_fp8") or []:
+            summary[f"prefill fp8 {p['shape']} b={p['b']} TFLOPs"] = p["TFLOPs"]
         if extras.get("recipe"):
             summary["recipe tokens_per_s"] = extras["recipe"]["tokens_per_s"]
             summary["recipe pct_hbm"] = extras["recipe"]["pct_hbm"]

@@ -464,6 +464,38 @@ MPW_API mpw_status mpw_qlinear_noalloc(const uint16_t* x, const uint8_t* packed,
                                        uint16_t* y, mpw_stream_t stream);
 
 /*
+ * FP8 (E4M3) prefill for codes of 4 or 5 bits.
+ * Pages: DynaQuant "Custom kernel architecture" (5-7-bit codes expanded to
+ * FP8 E4M3 and multiplied on FP8 tensor cores).  E4M3 holds integers exactly
+ * up to 16, so codes of b <= 5 (|q| <= 15) are exact; wider codes are
+ * refused (MPW_E_UNSUPPORTED_BITS).  The product needs x in E4M3 as well;
+ * this library's reading is the tutorial's symmetric per-channel formula per
+ * token, with E4M3's largest value 448 as max_int:
+ *   sx_m = fl32(max_k |x_mk| / 448) (a zero token: fl32(1 / 448)),
+ *   xq_mk = E4M3 of fl32(x_mk / sx_m), round to nearest even, saturating,
+ *   y_mn = bf16_rn(s_n * sx_m * sum_k xq_mk q_nk), fp32 accumulation.
+ * The result differs from mpw_qlinear's by the rounding of x to E4M3 (at most
+ * half an E4M3 step per element, 2^-4 relative); it is exact otherwise.
+ *
+ * mpw_quantize_x_fp8 -- x bf16 [M, K] -> xq E4M3 bytes [M, K] and sx fp32 [M].
+ *   K % 16 == 0; x and xq 16-byte aligned.
+ */
+MPW_API mpw_status mpw_quantize_x_fp8(const uint16_t* x, int64_t M, int64_t K, uint8_t* xq, float* sx,
+                                      mpw_stream_t stream);
+
+/*
+ * mpw_qlinear_fp8 -- y = sx * (xq @ q^T) * s on tcgen05 FP8 tensor cores
+ * (kind::f8f6f4), for any M (tiles of 256 tokens; M <= 16,776,960).
+ *   xq, sx   from mpw_quantize_x_fp8 (several linears may share them).
+ *   packed, scales  as produced by mpw_quantize_pack, bits 4 or 5, in
+ *            `layout` (MPW_LAYOUT_*; paired needs K % 32 == 0).
+ *   y        device, bf16 [M, N].  K % 16 == 0; xq and packed 16-byte aligned.
+ */
+MPW_API mpw_status mpw_qlinear_fp8(const uint8_t* xq, const float* sx, const uint8_t* packed, const float* scales,
+                                   int bits, int layout, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                                   mpw_stream_t stream);
+
+/*
  * mpw_gather_shards -- re-orders the gathered outputs of an output-row
  * (N) sharded linear into y.  No page describes tensor parallelism; the
  * partition is this library's: rank r of `world` owns weight rows
@@ -486,7 +518,7 @@ MPW_API mpw_status mpw_gather_shards(const uint16_t* blocks, int64_t world, int6
  *   other  the first bounded wait (2 s of waiting) inside a TMA / tensor-core
  *          kernel that gave up, as 100 * kernel + place: kernel 1 = per-tile
  *          decode, 2 = tensor-memory decode, 3 = prefill GEMM, 4 = stream-K
- *          decode; place 1 = x producer waiting for a free stage, 2 = x
+ *          decode, 5 = FP8 prefill GEMM; place 1 = x producer waiting for a free stage, 2 = x
  *          producer waiting for its last copies, 3 / 4 = the same for the
  *          weight (or combined) producer, 5 = consumer or MMA issuer waiting
  *          for a loaded stage, 6 = MMA issuer waiting for converted weights,

@@ -20,7 +20,7 @@ __all__ = [
     "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str", "allocate_bits", "allocation_frontier",
     "recipe_plan", "save_packed", "load_packed",
     "LAYOUTS", "workspace", "qlinear_workspace_bytes", "quantize_pack_groups", "qlinear_groups",
-    "gather_shards",
+    "gather_shards", "quantize_x_fp8", "qlinear_fp8",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmpw.so")
@@ -140,6 +140,10 @@ def _load():
     L.mpw_quantize_pack_groups.restype = c_int
     L.mpw_qlinear_groups.argtypes = [vp, vp, vp, c_int, i64, c_int, i64, i64, i64, vp, ctypes.c_uint, vp]
     L.mpw_qlinear_groups.restype = c_int
+    L.mpw_quantize_x_fp8.argtypes = [vp, i64, i64, vp, vp, vp]
+    L.mpw_quantize_x_fp8.restype = c_int
+    L.mpw_qlinear_fp8.argtypes = [vp, vp, vp, vp, c_int, c_int, i64, i64, i64, vp, vp]
+    L.mpw_qlinear_fp8.restype = c_int
     L.mpw_gather_shards.argtypes = [vp, i64, i64, i64, i64, vp, vp]
     L.mpw_gather_shards.restype = c_int
     L.mpw_device_error.argtypes = [ctypes.POINTER(i32)]
@@ -390,6 +394,45 @@ def qlinear_groups(x, packed, scales, bits: int, group: int, y=None, layout: str
     _check(lib.mpw_qlinear_groups(x.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits), int(group),
                                   LAYOUTS[layout], M, N, K, y.data_ptr(), flags, _stream(stream)),
            "mpw_qlinear_groups")
+    return y
+
+
+def quantize_x_fp8(x, xq=None, sx=None, stream=None):
+    """x bf16 [M, K] -> (xq uint8 [M, K] of E4M3 codes, sx fp32 [M]): the
+    per-token activations of the FP8 prefill (mpw_quantize_x_fp8)."""
+    import torch
+
+    _need(x, torch.bfloat16, "x", 2)
+    M, K = x.shape
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if sx is None:
+        sx = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _need(xq, torch.uint8, "xq", 2)
+    _need(sx, torch.float32, "sx", 1)
+    _check(lib.mpw_quantize_x_fp8(x.data_ptr(), M, K, xq.data_ptr(), sx.data_ptr(), _stream(stream)),
+           "mpw_quantize_x_fp8")
+    return xq, sx
+
+
+def qlinear_fp8(x, packed, scales, bits: int, y=None, layout: str = "canonical", xq=None, sx=None, stream=None):
+    """FP8 (E4M3) prefill linear for 4- and 5-bit codes (mpw_qlinear_fp8):
+    quantizes x per token unless (xq, sx) are given, then y bf16 [M, N]."""
+    import torch
+
+    _need(packed, torch.uint8, "packed", 2)
+    _need(scales, torch.float32, "scales", 1)
+    if xq is None or sx is None:
+        xq, sx = quantize_x_fp8(x, stream=stream)
+    M, K = xq.shape
+    N = packed.shape[0]
+    if packed.shape[1] != packed_row_bytes(K, bits):
+        raise ValueError("packed rows must be exactly packed_row_bytes(K, bits) long")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=packed.device)
+    _need(y, torch.bfloat16, "y")
+    _check(lib.mpw_qlinear_fp8(xq.data_ptr(), sx.data_ptr(), packed.data_ptr(), scales.data_ptr(), int(bits),
+                               LAYOUTS[layout], M, N, K, y.data_ptr(), _stream(stream)), "mpw_qlinear_fp8")
     return y
 
 

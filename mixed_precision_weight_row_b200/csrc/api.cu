@@ -218,6 +218,28 @@ mpw_status mpw_qlinear_groups(const uint16_t* x, const uint8_t* packed, const fl
                                       reinterpret_cast<cudaStream_t>(stream), flags));
 }
 
+mpw_status mpw_quantize_x_fp8(const uint16_t* x, int64_t M, int64_t K, uint8_t* xq, float* sx, mpw_stream_t stream) {
+  if (x == nullptr || xq == nullptr || sx == nullptr || M < 1 || K < 16) return MPW_E_INVALID_ARG;
+  if (M > 0x7fffffff || K > 0x3fffffff || K % 16 != 0) return MPW_E_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(xq, 16) || !aligned(sx, 4)) return MPW_E_MISALIGNED;
+  return from_cuda(launch_quantize_x_fp8(x, M, K, xq, sx, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mpw_status mpw_qlinear_fp8(const uint8_t* xq, const float* sx, const uint8_t* packed, const float* scales, int bits,
+                           int layout, int64_t M, int64_t N, int64_t K, uint16_t* y, mpw_stream_t stream) {
+  if (bits != 4 && bits != 5) return MPW_E_UNSUPPORTED_BITS;
+  if (xq == nullptr || sx == nullptr || packed == nullptr || scales == nullptr || y == nullptr || M < 1 || N < 1 ||
+      K < 16)
+    return MPW_E_INVALID_ARG;
+  if (M > 0x7fffffff || N > 0x7fffffff || K > 0x3fffffff || K % 16 != 0 || !layout_ok(layout)) return MPW_E_INVALID_ARG;
+  if (layout == MPW_LAYOUT_PAIRED && K % 32 != 0) return MPW_E_INVALID_ARG;
+  if ((M + 255) / 256 > 65535) return MPW_E_INVALID_ARG;
+  if (!aligned(xq, 16) || !aligned(packed, 16) || !aligned(sx, 4) || !aligned(scales, 4) || !aligned(y, 2))
+    return MPW_E_MISALIGNED;
+  return from_cuda(launch_gemm_fp8(xq, sx, packed, scales, bits, layout, M, N, K, y,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
 mpw_status mpw_gather_shards(const uint16_t* blocks, int64_t world, int64_t M, int64_t Nl, int64_t N, uint16_t* y,
                              mpw_stream_t stream) {
   if (blocks == nullptr || y == nullptr || world < 1 || M < 1 || Nl < 1 || N < 1) return MPW_E_INVALID_ARG;

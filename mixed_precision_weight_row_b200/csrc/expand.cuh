@@ -300,6 +300,26 @@ __device__ __forceinline__ void gemm_expand_group(const uint32_t (&w)[B + 1],
   gemm_all<B, PAIRED>(w, v, std::make_integer_sequence<int, 16>{});
 }
 
+// Bits of codes 2I and 2I+1 of a 32-code group at bit 0 of the low and of the
+// high half of the result (the higher bits of each half are the neighbours'),
+// for either layout.
+template <int B, bool PAIRED, int I>
+__device__ __forceinline__ uint32_t pair_window(const uint32_t (&w)[B + 1]) {
+  if constexpr (PAIRED) {
+    constexpr int o = I * B;
+    constexpr int h = o >> 4, r = o & 15;
+    if constexpr (r + B <= 16) {
+      return r == 0 ? w[h] : (w[h] >> r);
+    } else {
+      constexpr uint32_t sel = ((1u << (16 - r)) - 1u) * 0x10001u;
+      return ((w[h] >> r) & sel) | ((w[h + 1] << (16 - r)) & ~sel);
+    }
+  } else {
+    const uint32_t t = window<B>(w, 2 * I * B);   // code 2I at bit 0, code 2I+1 at bit B
+    return merge_halves(t, t << (16 - B));
+  }
+}
+
 __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
   asm volatile(

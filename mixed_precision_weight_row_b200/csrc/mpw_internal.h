@@ -140,6 +140,14 @@ cudaError_t launch_gemv_groups(const uint16_t* x, const uint8_t* packed, const f
 cudaError_t launch_gather_shards(const uint16_t* blocks, int64_t M, int64_t Nl, int64_t N, uint16_t* y,
                                  cudaStream_t stream);
 
+// gemm_fp8.cu: per-token E4M3 activations (K % 16 == 0) and the E4M3 prefill
+// GEMM for codes of 4 or 5 bits.
+cudaError_t launch_quantize_x_fp8(const uint16_t* x, int64_t M, int64_t K, uint8_t* xq, float* sx,
+                                  cudaStream_t stream);
+cudaError_t launch_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* packed, const float* scales,
+                            int bits, int layout, int64_t M, int64_t N, int64_t K, uint16_t* y,
+                            cudaStream_t stream);
+
 // gemm.cu: tcgen05 prefill GEMM; returns cudaErrorNotSupported for shapes it
 // does not take (the caller then uses the GEMV path).
 cudaError_t launch_gemm(const uint16_t* x, const uint8_t* packed, const float* scales,

@@ -66,7 +66,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 
 // Codes a wait that gives up leaves in the device error word:
 // 100 * kernel + place.  The first one stays until the word is read.
-enum WaitKernel : int32_t { kWaitGemvTma = 1, kWaitGemvTc = 2, kWaitGemm = 3, kWaitGemvSk = 4 };
+enum WaitKernel : int32_t { kWaitGemvTma = 1, kWaitGemvTc = 2, kWaitGemm = 3, kWaitGemvSk = 4, kWaitGemmFp8 = 5 };
 enum WaitPlace : int32_t {
   kWaitXEmpty = 1,    // x producer: a free x stage
   kWaitXTail = 2,     // x producer: its last copies landed
@@ -227,6 +227,18 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f8f6f4 (operand types in idesc,
+// fp32 accumulator).
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives once on the mbarrier when every tcgen05.mma issued so far by this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -251,6 +263,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4)                                    // D format: f32
          | (1u << 7)                                  // A format: bf16
          | (1u << 10)                                 // B format: bf16
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
+}
+
+// Instruction descriptor: E4M3 x E4M3 -> fp32 (kind::f8f6f4), both operands
+// K-major (format code 0 = E4M3 for A and B).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                    // D format: f32
+         | (0u << 7)                                  // A format: E4M3
+         | (0u << 10)                                 // B format: E4M3
          | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }

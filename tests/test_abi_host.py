@@ -260,3 +260,23 @@ def test_group_entry_points_validation():
     assert ql(0, A16B, A16, 5, 128, 0, 1, 16, 256, A16, 0, 0) == mpw.MPW_E_INVALID_ARG
     assert ql(A16, A16B, A16, 5, 128, 0, 1, 16, 256, A16, 2, 0) == mpw.MPW_E_INVALID_ARG   # y_unshared alone
     assert ql(A16, A16B, A16, 5, 128, 0, 1, 16, 256, A16, 4, 0) == mpw.MPW_E_INVALID_ARG   # unknown flag
+
+
+def test_fp8_entry_points_validation():
+    L = mpw.lib
+    # x, M, K, xq, sx, stream
+    assert L.mpw_quantize_x_fp8(0, 4, 64, A16B, A16, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_quantize_x_fp8(A16, 0, 64, A16B, A16, 0) == mpw.MPW_E_INVALID_ARG
+    assert L.mpw_quantize_x_fp8(A16, 4, 72, A16B, A16, 0) == mpw.MPW_E_INVALID_ARG     # K % 16
+    assert L.mpw_quantize_x_fp8(A16 + 2, 4, 64, A16B, A16, 0) == mpw.MPW_E_MISALIGNED
+    assert L.mpw_quantize_x_fp8(A16, 4, 64, A16B + 8, A16, 0) == mpw.MPW_E_MISALIGNED
+    q8 = L.mpw_qlinear_fp8
+    # xq, sx, packed, scales, bits, layout, M, N, K, y, stream
+    for b in (3, 6, 8, 15):
+        assert q8(A16, A16, A16B, A16, b, 0, 4, 16, 64, A16, 0) == mpw.MPW_E_UNSUPPORTED_BITS
+    assert q8(A16, A16, A16B, A16, 5, 0, 4, 16, 72, A16, 0) == mpw.MPW_E_INVALID_ARG      # K % 16
+    assert q8(A16, A16, A16B, A16, 5, 1, 4, 16, 80, A16, 0) == mpw.MPW_E_INVALID_ARG      # paired K % 32
+    assert q8(A16, A16, A16B, A16, 5, 2, 4, 16, 64, A16, 0) == mpw.MPW_E_INVALID_ARG      # layout
+    assert q8(A16 + 8, A16, A16B, A16, 5, 0, 4, 16, 64, A16, 0) == mpw.MPW_E_MISALIGNED
+    assert q8(A16, A16, A16B + 8, A16, 5, 0, 4, 16, 64, A16, 0) == mpw.MPW_E_MISALIGNED
+    assert q8(0, A16, A16B, A16, 5, 0, 4, 16, 64, A16, 0) == mpw.MPW_E_INVALID_ARG
