@@ -59,7 +59,7 @@ def peaks():
 
 # Sources whose change invalidates a committed DRAM-traffic figure for the
 # decode kernel that the headline times.
-TMA_GEMV_SOURCES = ["gemv_tma.cu", "expand.cuh", "tc_ptx.cuh"]
+TMA_GEMV_SOURCES = ["gemv_tma.cuh", "gemv_tma.cu", "expand.cuh", "tc_ptx.cuh"]
 
 
 def kernel_source_hash(names):
@@ -675,14 +675,14 @@ def run_case(args):
     import workloads as wl
 
     b, M = args.bits, args.M
-    if args.case in ("decode", "quantize"):
+    if args.case in ("decode", "quantize", "groups"):
         c = wl.DECODE
         W = torch.from_numpy(wl.gen_weight(c["N"], c["K"], c["sigma"], c["w_seed"], c["outlier_frac"],
                                            c["outlier_scale"])).cuda()
     elif args.case in ("gate", "down"):
         _, N, K = dict((n, (n, a, k)) for n, a, k in wl.MLP27B["shapes"])[args.case]
         W = wl.gen_weight_torch(N, K, wl.MLP27B["sigma"], 17 + N)
-    elif args.case == "prefill":
+    elif args.case in ("prefill", "prefill_fp8"):
         _, N, K = wl.PREFILL["shapes"][0]
         W = wl.gen_weight_torch(N, K, wl.PREFILL["sigma"], 11 + N)
         M = wl.PREFILL["M"]
@@ -700,6 +700,21 @@ def run_case(args):
     elif args.case == "quantize":
         for _ in range(args.launches):
             mpw.quantize_pack(W, b)
+    elif args.case == "groups":
+        packed, scales = mpw.quantize_pack_groups(W, b, args.group)
+        if args.layout != "canonical":
+            packed = mpw.repack(packed, W.shape[1], b, "canonical", args.layout)
+        x = wl.gen_x(M, W.shape[1], 1).cuda()
+        for _ in range(args.launches):
+            mpw.qlinear_groups(x, packed, scales, b, args.group, layout=args.layout)
+    elif args.case == "prefill_fp8":
+        packed, scales = mpw.quantize_pack(W, b)
+        if args.layout != "canonical":
+            packed = mpw.repack(packed, W.shape[1], b, "canonical", args.layout)
+        x = wl.gen_x(M, W.shape[1], 1).cuda()
+        xq, sx = mpw.quantize_x_fp8(x)
+        for _ in range(args.launches):
+            mpw.qlinear_fp8(x, packed, scales, b, layout=args.layout, xq=xq, sx=sx)
     else:
         packed, scales = mpw.quantize_pack(W, b)
         if args.layout != "canonical":
@@ -734,13 +749,15 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
-    ap.add_argument("--case", choices=["decode", "gate", "down", "prefill", "recipe", "quantize"],
+    ap.add_argument("--case", choices=["decode", "gate", "down", "prefill", "recipe", "quantize", "groups",
+                                       "prefill_fp8"],
                     default=None, help="profiling target: run a few launches of one kernel, print nothing")
     ap.add_argument("--bits", type=int, default=HEADLINE_BITS, help="bit width for --case")
     ap.add_argument("--M", type=int, default=1, help="tokens for --case")
     ap.add_argument("--layout", choices=["canonical", "paired"], default="paired",
                     help="packed layout the decode and prefill kernels read (repacked outside the timed region)")
     ap.add_argument("--launches", type=int, default=5, help="launches for --case")
+    ap.add_argument("--group", type=int, default=128, help="group size for --case groups")
     ap.add_argument("--quick", action="store_true",
                     help="headline and e2e only (no sweep, extras or CPU baseline)")
     args = ap.parse_args(argv)
