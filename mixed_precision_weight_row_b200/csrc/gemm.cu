@@ -7,7 +7,9 @@
 // closing note: prefill is compute-bound.
 //
 // One CTA computes a 128-row (W) x 256-token (x) tile of y^T with
-// tcgen05.mma.cta_group::1.kind::f16, M=128, N=256, K=16:
+// tcgen05.mma.cta_group::1.kind::f16, M=128, N=256, K=16 (192-token tiles,
+// N=192, on shapes where 256-token tiles would leave a mostly empty last
+// wave of CTAs):
 //   * Packed weights move in blocks of 128 codes (16*B bytes per row), one 2D
 //     TMA per block ({16*B bytes x 128 rows}) into a 3-stage ring; rows past
 //     N and bytes past the row read as zeros.  The converters read a row's
@@ -45,20 +47,21 @@ namespace {
 using namespace dec;
 
 constexpr int BM = 128;          // weight rows per CTA (MMA M)
-constexpr int BN = 256;          // tokens per CTA (MMA N)
 constexpr int BK = 64;           // codes per x stage (one 128-byte swizzle atom of bf16)
 constexpr int WB = 128;          // codes per weight block
 constexpr int SW = 3;            // weight stages in shared memory
 constexpr int kThreads = 384;    // 12 warps
 constexpr int kConvWarp0 = 4;    // first converter warp
-constexpr uint32_t kXStageBytes = BN * BK * 2;   // 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCols = BN;                // fp32 accumulator columns
 
-template <int B>
+// BN: tokens per CTA (the MMA's N), 256 or 192 (chosen per shape so that the
+// tiles fill the SMs in whole waves).
+template <int B, int BN>
 struct GemmCode {
+  static constexpr uint32_t kXStageBytes = BN * BK * 2;   // 32 KB at BN = 256
+  static constexpr uint32_t kAccCols = BN;                // fp32 accumulator columns
   // x stages in shared memory: as many as fit beside the weight stages
-  static constexpr int SX = B <= 8 ? 5 : 4;
+  static constexpr int SX = BN == 256 ? (B <= 8 ? 5 : 4) : (B <= 8 ? 6 : 5);
   static constexpr int P = GemmParts<B>::parts;              // MMAs per k-step
   static constexpr uint32_t ACOLS = 64u * P;                 // tensor-memory columns per A stage
   static constexpr int SA = static_cast<int>((kTmemCols - kAccCols) / ACOLS);
@@ -78,15 +81,17 @@ struct GemmCode {
 };
 
 
-template <int B, bool PAIRED>
+template <int B, bool PAIRED, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
             const float* __restrict__ scales, uint16_t* __restrict__ y, int M, int N, int K, int rb,
             int32_t* err) {
-  using C = GemmCode<B>;
+  using C = GemmCode<B, BN>;
   constexpr int P = C::P;
   constexpr int SA = C::SA;
   constexpr int SX = C::SX;
+  constexpr uint32_t kXStageBytes = C::kXStageBytes;
+  constexpr uint32_t kAccCols = C::kAccCols;
   extern __shared__ uint8_t gsmem_raw[];
   const uint32_t raw = ptx::smem_addr(gsmem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;       // 1024-aligned for the 128-byte swizzle
@@ -105,8 +110,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
   const uint32_t acc_full = bar0 + 8u * (2 * SX + 2 * SW + 2 * SA);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BM;
-  const int m0 = blockIdx.y * BN;
+  // token tiles run fastest: the CTAs resident together share weight rows,
+  // which then come from L2 after the first of them has read them
+  const int m0 = blockIdx.x * BN;
+  const int n0 = blockIdx.y * BM;
   const int KB = (K + BK - 1) / BK;      // x stages
   const int WBs = (K + WB - 1) / WB;     // weight blocks
 
@@ -266,10 +273,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
   }
 }
 
-template <int B, bool PAIRED>
+template <int B, bool PAIRED, int BN>
 cudaError_t run_gemm(const uint16_t* x, const uint8_t* packed, const float* scales, int64_t M,
                      int64_t N, int64_t K, uint16_t* y, int32_t* err, cudaStream_t stream) {
-  using C = GemmCode<B>;
+  using C = GemmCode<B, BN>;
   auto encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap;
@@ -292,31 +299,51 @@ cudaError_t run_gemm(const uint16_t* x, const uint8_t* packed, const float* scal
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = gemm_kernel<B, PAIRED>;
+  auto kern = gemm_kernel<B, PAIRED, BN>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>((N + BM - 1) / BM), static_cast<unsigned>((M + BN - 1) / BN));
+  const dim3 grid(static_cast<unsigned>((M + BN - 1) / BN), static_cast<unsigned>((N + BM - 1) / BM));
   kern<<<grid, kThreads, C::SMEM, stream>>>(tmap, tmap_w, scales, y, static_cast<int>(M), static_cast<int>(N),
                                             static_cast<int>(K), static_cast<int>(rb), err);
   return cudaGetLastError();
+}
+
+// Fraction of the SMs' tile slots that do useful work with token tiles of
+// bn: whole waves of one CTA per SM, less the padding of the last token tile.
+double tile_efficiency(int64_t M, int64_t N, int bn, int sms) {
+  const int64_t mt = (M + bn - 1) / bn, tiles = mt * ((N + BM - 1) / BM);
+  const int64_t rounds = (tiles + sms - 1) / sms;
+  return static_cast<double>(tiles) / static_cast<double>(rounds * sms) *
+         static_cast<double>(M) / static_cast<double>(mt * bn);
+}
+
+template <int B, bool PAIRED>
+cudaError_t gemm_bn(const uint16_t* x, const uint8_t* packed, const float* scales, int64_t M, int64_t N,
+                    int64_t K, uint16_t* y, int32_t* err, cudaStream_t stream) {
+  // 256-token tiles convert each weight block for more tokens; 192-token
+  // tiles only when they fill the SMs clearly better
+  const int sms = device_info().num_sms;
+  if (tile_efficiency(M, N, 192, sms) > tile_efficiency(M, N, 256, sms) + 0.05)
+    return run_gemm<B, PAIRED, 192>(x, packed, scales, M, N, K, y, err, stream);
+  return run_gemm<B, PAIRED, 256>(x, packed, scales, M, N, K, y, err, stream);
 }
 
 template <bool PAIRED>
 cudaError_t gemm_layout(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int64_t M,
                         int64_t N, int64_t K, uint16_t* y, int32_t* err, cudaStream_t stream) {
   switch (bits) {
-    case 4: return run_gemm<4, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 5: return run_gemm<5, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 6: return run_gemm<6, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 7: return run_gemm<7, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 8: return run_gemm<8, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 9: return run_gemm<9, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 10: return run_gemm<10, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 11: return run_gemm<11, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 12: return run_gemm<12, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 13: return run_gemm<13, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 14: return run_gemm<14, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
-    case 15: return run_gemm<15, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 4: return gemm_bn<4, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 5: return gemm_bn<5, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 6: return gemm_bn<6, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 7: return gemm_bn<7, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 8: return gemm_bn<8, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 9: return gemm_bn<9, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 10: return gemm_bn<10, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 11: return gemm_bn<11, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 12: return gemm_bn<12, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 13: return gemm_bn<13, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 14: return gemm_bn<14, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
+    case 15: return gemm_bn<15, PAIRED>(x, packed, scales, M, N, K, y, err, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -325,7 +352,7 @@ cudaError_t gemm_layout(const uint16_t* x, const uint8_t* packed, const float* s
 
 bool gemm_supported(int64_t M, int64_t N, int64_t K) {
   // TMA needs the x row stride (K * 2 bytes) to be a multiple of 16 bytes.
-  return K % 8 == 0 && M >= 1 && N >= 1 && (M + BN - 1) / BN <= 65535;
+  return K % 8 == 0 && M >= 1 && N >= 1 && (N + BM - 1) / BM <= 65535;
 }
 
 cudaError_t launch_gemm(const uint16_t* x, const uint8_t* packed, const float* scales, int bits, int layout,

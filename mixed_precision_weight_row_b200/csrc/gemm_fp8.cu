@@ -43,21 +43,22 @@ namespace {
 using namespace dec;
 
 constexpr int BM = 128;          // weight rows per CTA (MMA M)
-constexpr int BN = 256;          // tokens per CTA (MMA N)
 constexpr int BK = 128;          // codes per block and per x stage (128 bytes of E4M3)
 constexpr int SX = 4;            // x stages
 constexpr int SW = 4;            // weight stages
 constexpr int kThreads = 384;
 constexpr int kConvWarp0 = 4;
-constexpr uint32_t kXStageBytes = BN * BK;               // 32 KB
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCols = BN;                        // fp32 accumulator columns
 constexpr uint32_t kACols = BK / 4;                      // one A stage: 128 bytes per row
-constexpr int SA = static_cast<int>((kTmemCols - kAccCols) / kACols);
 constexpr float kE4M3Max = 448.0f;
 
-template <int B>
+// BN: tokens per CTA (the MMA's N), 256 or 192 (chosen per shape so that the
+// tiles fill the SMs in whole waves).
+template <int B, int BN>
 struct F8Code {
+  static constexpr uint32_t kXStageBytes = BN * BK;      // 32 KB at BN = 256
+  static constexpr uint32_t kAccCols = BN;               // fp32 accumulator columns
+  static constexpr int SA = static_cast<int>((kTmemCols - kAccCols) / kACols);
   static constexpr uint32_t PITCH = 16u * B;
   static constexpr uint32_t WSTAGE = BM * PITCH;
   static constexpr CUtensorMapSwizzle WSWZ = B == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
@@ -97,12 +98,15 @@ __device__ __forceinline__ void e4m3_group(const uint32_t (&w)[B + 1], uint32_t 
   e4m3_all<B, PAIRED>(w, o, std::make_integer_sequence<int, 8>{});
 }
 
-template <int B, bool PAIRED>
+template <int B, bool PAIRED, int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                 const float* __restrict__ scales, const float* __restrict__ sx, uint16_t* __restrict__ y, int M,
                 int N, int K, int32_t* err) {
-  using C = F8Code<B>;
+  using C = F8Code<B, BN>;
+  constexpr uint32_t kXStageBytes = C::kXStageBytes;
+  constexpr uint32_t kAccCols = C::kAccCols;
+  constexpr int SA = C::SA;
   extern __shared__ uint8_t fsmem_raw[];
   __shared__ float sx_s[BN];
   const uint32_t raw = ptx::smem_addr(fsmem_raw);
@@ -123,8 +127,9 @@ gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constan
   constexpr int32_t kW = ptx::kWaitGemmFp8;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BM;
-  const int m0 = blockIdx.y * BN;
+  // token tiles run fastest (CTAs resident together share weight rows)
+  const int m0 = blockIdx.x * BN;
+  const int n0 = blockIdx.y * BM;
   const int KB = (K + BK - 1) / BK;      // blocks (one x stage and one weight block each)
 
   if (threadIdx.x < BN) sx_s[threadIdx.x] = m0 + static_cast<int>(threadIdx.x) < M ? sx[m0 + threadIdx.x] : 0.0f;
@@ -333,10 +338,10 @@ quantize_x_fp8_kernel(const uint16_t* __restrict__ x, int K, uint8_t* __restrict
   }
 }
 
-template <int B, bool PAIRED>
+template <int B, bool PAIRED, int BN>
 cudaError_t run_fp8(const uint8_t* xq, const float* sx, const uint8_t* packed, const float* scales, int64_t M,
                     int64_t N, int64_t K, uint16_t* y, int32_t* err, cudaStream_t stream) {
-  using C = F8Code<B>;
+  using C = F8Code<B, BN>;
   auto encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap;
@@ -359,13 +364,31 @@ cudaError_t run_fp8(const uint8_t* xq, const float* sx, const uint8_t* packed, c
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = gemm_fp8_kernel<B, PAIRED>;
+  auto kern = gemm_fp8_kernel<B, PAIRED, BN>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>((N + BM - 1) / BM), static_cast<unsigned>((M + BN - 1) / BN));
+  const dim3 grid(static_cast<unsigned>((M + BN - 1) / BN), static_cast<unsigned>((N + BM - 1) / BM));
   kern<<<grid, kThreads, C::SMEM, stream>>>(tmap, tmap_w, scales, sx, y, static_cast<int>(M), static_cast<int>(N),
                                             static_cast<int>(K), err);
   return cudaGetLastError();
+}
+
+// Fraction of the SMs' tile slots that do useful work with token tiles of
+// bn (whole waves of one CTA per SM, less the padding of the last token tile).
+double fp8_tile_efficiency(int64_t M, int64_t N, int bn, int sms) {
+  const int64_t mt = (M + bn - 1) / bn, tiles = mt * ((N + BM - 1) / BM);
+  const int64_t rounds = (tiles + sms - 1) / sms;
+  return static_cast<double>(tiles) / static_cast<double>(rounds * sms) *
+         static_cast<double>(M) / static_cast<double>(mt * bn);
+}
+
+template <int B, bool PAIRED>
+cudaError_t fp8_bn(const uint8_t* xq, const float* sx, const uint8_t* packed, const float* scales, int64_t M,
+                   int64_t N, int64_t K, uint16_t* y, int32_t* err, cudaStream_t stream) {
+  const int sms = device_info().num_sms;
+  if (fp8_tile_efficiency(M, N, 192, sms) > fp8_tile_efficiency(M, N, 256, sms) + 0.05)
+    return run_fp8<B, PAIRED, 192>(xq, sx, packed, scales, M, N, K, y, err, stream);
+  return run_fp8<B, PAIRED, 256>(xq, sx, packed, scales, M, N, K, y, err, stream);
 }
 
 }  // namespace
@@ -382,11 +405,11 @@ cudaError_t launch_gemm_fp8(const uint8_t* xq, const float* sx, const uint8_t* p
   int32_t* err = device_error_word();
   const bool paired = layout == kLayoutPaired;
   if (bits == 4)
-    return paired ? run_fp8<4, true>(xq, sx, packed, scales, M, N, K, y, err, stream)
-                  : run_fp8<4, false>(xq, sx, packed, scales, M, N, K, y, err, stream);
+    return paired ? fp8_bn<4, true>(xq, sx, packed, scales, M, N, K, y, err, stream)
+                  : fp8_bn<4, false>(xq, sx, packed, scales, M, N, K, y, err, stream);
   if (bits == 5)
-    return paired ? run_fp8<5, true>(xq, sx, packed, scales, M, N, K, y, err, stream)
-                  : run_fp8<5, false>(xq, sx, packed, scales, M, N, K, y, err, stream);
+    return paired ? fp8_bn<5, true>(xq, sx, packed, scales, M, N, K, y, err, stream)
+                  : fp8_bn<5, false>(xq, sx, packed, scales, M, N, K, y, err, stream);
   return cudaErrorInvalidValue;
 }
 
