@@ -165,7 +165,7 @@ constexpr int min_ctas_for() {
 // one group, so a chunk's products are summed on their own and join the
 // accumulator multiplied by the group's scale (fp32).
 template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false>
-__global__ void __launch_bounds__(kThreads, GRP ? min_ctas<B, NT>() : min_ctas_for<B, NT, NSQ, PAIRED>())
+__global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, NSQ, PAIRED>())
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                 int M, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
                 int flags, int32_t* err, int gstride, int gshift) {
