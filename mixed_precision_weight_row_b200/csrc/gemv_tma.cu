@@ -9,8 +9,10 @@ namespace {
 template <int B, bool PAIRED>
 cudaError_t tma_bits(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
                      uint16_t* y, bool norm, bool pdl, int flags, int32_t* err, cudaStream_t stream) {
-  if (norm && M == 1) return run_tma<B, 1, 1, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  // one token: the token count is a compile-time constant
+  if (norm && M == 1) return run_tma<B, 1, 1, PAIRED, false, 1>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
   if (norm) return run_tma<B, 1, kNormMaxM, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  if (M == 1) return run_tma<B, 1, 0, PAIRED, false, 1>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
   if (M <= 8) return run_tma<B, 1, 0, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
   if (M <= 16) return run_tma<B, 2, 0, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
   return run_tma<B, 4, 0, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);

@@ -164,11 +164,14 @@ constexpr int min_ctas_for() {
 // (scales [N, gstride]) instead of one per row: each 128-code chunk lies in
 // one group, so a chunk's products are summed on their own and join the
 // accumulator multiplied by the group's scale (fp32).
-template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false>
+// MC: the number of tokens when it is fixed at compile time (1 for the one-
+// token decode step), else 0 and M is read at run time.
+template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0>
 __global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, NSQ, PAIRED>())
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-                int M, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
+                int M_, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
                 int flags, int32_t* err, int gstride, int gshift) {
+  const int M = MC > 0 ? MC : M_;
   static_assert(!GRP || NSQ == 0, "group scales with the plain input only");
   constexpr int P = dec_parts<B, PAIRED>();
   constexpr bool NORM = NSQ > 0;
@@ -392,9 +395,15 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
       if (!ptx::mbar_wait(full(slot), phase, err, ptx::wait_code(ptx::kWaitGemvTma, ptx::kWaitFull))) break;
       const uint8_t* st = tsmem + st_off;
       const int c_first = cb + kSC * s + warp * kCH;
+      if (cb + kSC * (s + 1) <= ce) {
+        // a whole stage: every chunk is in range
 #pragma unroll
-      for (int h = 0; h < kCH; ++h)
-        chunk(st, warp * kCH + h, c_first + h, c_first + h < ce, h == kCH - 1, empty(slot));
+        for (int h = 0; h < kCH; ++h) chunk(st, warp * kCH + h, c_first + h, true, h == kCH - 1, empty(slot));
+      } else {
+#pragma unroll
+        for (int h = 0; h < kCH; ++h)
+          chunk(st, warp * kCH + h, c_first + h, c_first + h < ce, h == kCH - 1, empty(slot));
+      }
       st_off += st_bytes;
       if (++slot == S) {
         slot = 0;
@@ -543,7 +552,8 @@ int cluster_size(int tiles, int chunks, int num_sms) {
 }
 
 // gstride, gshift: group scales (GRP; see the kernel), else unused.
-template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false>
+// MC: as for the kernel (M must then equal MC).
+template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0>
 cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
                     uint16_t* y, bool pdl, int flags, int32_t* err, cudaStream_t stream, int gstride = 0,
                     int gshift = 0) {
@@ -596,14 +606,15 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP>;
+  auto kern = gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC>;
   const int tiles = (N + 15) / 16;
   const int kc = cluster_size(tiles, chunks, device_info().num_sms);
   const int per_cta = ((chunks + kc - 1) / kc + kSC - 1) / kSC;
   // resident CTAs per SM that registers and static shared memory allow
   static const int ctas_by_regs = [] {
     int n = 0;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP>, kThreads, 0) ==
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC>, kThreads,
+                                                         0) ==
                    cudaSuccess
                ? n
                : 0;
