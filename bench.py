@@ -921,7 +921,8 @@ def main(argv=None):
         extras["summary"] = summary
 
     traffic = profile_traffic(f"gemv_tma_decode_b6_m1_{lay}.json", TMA_GEMV_SOURCES)
-    roof = {"bound": "hbm", "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,0,{str(lay == 'paired').lower()}>",
+    roof = {"bound": "hbm",
+            "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,0,{str(lay == 'paired').lower()},false,1>",
             "achieved": round(achieved, 1) if achieved is not None else None,
             "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / pk["hbm_gbs"], 4) if achieved is not None else None,
