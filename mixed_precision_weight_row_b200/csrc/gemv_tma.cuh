@@ -75,10 +75,10 @@ constexpr int kXReady = 1;              // flags: x is not written by the preced
 constexpr int kStageBoxes = 2;          // flags: one 3D TMA per stage and operand
 constexpr int kYFree = 4;               // flags: no call of the run touches y
 
-// Bytes of one stage: kSC weight chunks (16 rows x 16*B bytes) followed by
-// kSC x chunks (M tokens x 128 bf16).
-__host__ __device__ constexpr uint32_t stage_bytes(int B, int M) {
-  return static_cast<uint32_t>(kSC) * 256u * static_cast<uint32_t>(B + M);
+// Bytes of one stage: kSC weight chunks (16*RT rows x 16*B bytes) followed
+// by kSC x chunks (M tokens x 128 bf16).
+__host__ __device__ constexpr uint32_t stage_bytes(int B, int M, int RT = 1) {
+  return static_cast<uint32_t>(kSC) * 256u * static_cast<uint32_t>(B * RT + M);
 }
 
 // Ring depth.  When the grid fits on the SMs in one wave, a CTA whose whole
@@ -91,13 +91,13 @@ __host__ __device__ constexpr uint32_t stage_bytes(int B, int M) {
 // MPW_GEMV_RING_KB replaces the rule by a fixed budget (tuning aid).
 constexpr uint32_t kWholeSlice = 64u * 1024u;
 
-int ring_stages(int B, int M, int stages_per_cta, bool few_ctas, int ctas_by_regs, uint32_t fixed) {
+int ring_stages(int B, int M, int stages_per_cta, bool few_ctas, int ctas_by_regs, uint32_t fixed, int RT = 1) {
   static const uint32_t budget = [] {
     const char* e = tuning_env("MPW_GEMV_RING_KB");
     const int v = e ? atoi(e) : 0;
     return v >= 8 && v <= 192 ? static_cast<uint32_t>(v) * 1024u : 0u;
   }();
-  const uint32_t st = stage_bytes(B, M);
+  const uint32_t st = stage_bytes(B, M, RT);
   int s;
   if (budget != 0) {
     s = static_cast<int>(budget / st);
@@ -166,7 +166,11 @@ constexpr int min_ctas_for() {
 // accumulator multiplied by the group's scale (fp32).
 // MC: the number of tokens when it is fixed at compile time (1 for the one-
 // token decode step), else 0 and M is read at run time.
-template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0>
+// RT: 16-row tiles per CTA.  The RT tiles share each stage's x chunks (x is
+// loaded once for 16*RT rows instead of once per 16), which matters when
+// several tokens make x as large as the weights; consumer warp w takes tile
+// w % RT and 2*RT of the stage's chunks.
+template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0, int RT = 1>
 __global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, NSQ, PAIRED>())
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                 int M_, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
@@ -176,10 +180,12 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
   constexpr int P = dec_parts<B, PAIRED>();
   constexpr bool NORM = NSQ > 0;
   constexpr int NS = NSQ > 0 ? NSQ : 1;
-  constexpr uint32_t kWChunk = 256u * B;        // 16 rows x 16*B bytes
+  static_assert(RT == 1 || RT == 2 || RT == 4, "row tiles per CTA");
+  constexpr uint32_t kWChunk = 256u * B * RT;   // 16*RT rows x 16*B bytes
+  constexpr int kCHW = kCH * RT;                // chunks per consumer warp and stage
   const uint32_t x_chunk = 256u * M;            // M tokens x 128 bf16
   const uint32_t w_part = kSC * kWChunk;
-  const uint32_t st_bytes = stage_bytes(B, M);
+  const uint32_t st_bytes = stage_bytes(B, M, RT);
   // dynamic: the ring (S stages), then, in clusters, the partial sums of the
   // cluster's CTAs
   extern __shared__ __align__(128) uint8_t tsmem[];
@@ -188,7 +194,8 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
   __shared__ float ss_red[kCW][NS];
   __shared__ float cl_ss[8][NS];
   __shared__ __align__(16) uint4 zero_x[4];   // x fragment of lanes without a token
-  auto cl_red = reinterpret_cast<float (*)[NT][32][4]>(tsmem + static_cast<uint32_t>(S) * stage_bytes(B, M));
+  // cluster partial sums: [cluster rank][row tile][NT][32][4]
+  auto cl_red = reinterpret_cast<float (*)[RT][NT][32][4]>(tsmem + static_cast<uint32_t>(S) * stage_bytes(B, M, RT));
 
   if (flags & kXReady) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cg::cluster_group cluster = cg::this_cluster();
@@ -202,7 +209,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
   const int cb = cr * cpc;
   const int ce = min(chunks, cb + cpc);
   const int n_stages = ce > cb ? (ce - cb + kSC - 1) / kSC : 0;
-  const int r0 = tile * 16;
+  const int r0 = tile * 16 * RT;
   const uint32_t base = ptx::smem_addr(tsmem);
   const uint32_t bar0 = ptx::smem_addr(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
@@ -293,9 +300,11 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
     uint32_t x_lane[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) x_lane[nt] = (g + 8 * nt) * 256 + tig * 64;
-    const uint32_t w_lane = tig * 4 * B + g * 16 * B;
+    // this warp's row tile and its share of each stage's chunks
+    const int rt = warp % RT, wsub = warp / RT;
+    const uint32_t w_lane = rt * 256u * B + tig * 4 * B + g * 16 * B;
     // rows of this lane's accumulator entries (0, 1: row g; 2, 3: row g + 8)
-    const int row_a = r0 + g, row_b = r0 + g + 8;
+    const int row_a = r0 + 16 * rt + g, row_b = row_a + 8;
 
     // One chunk (global index c): B words of rows g and g+8, the x fragment
     // of token g, expand, (release the stage after its last chunk), MMAs.
@@ -323,8 +332,9 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
           xw[nt][4 * q] = v.x; xw[nt][4 * q + 1] = v.y; xw[nt][4 * q + 2] = v.z; xw[nt][4 * q + 3] = v.w;
         }
       }
-      if (NORM && active) {
-        // squares of x for the rms scale: 4 of the chunk's 128 values per lane
+      if (NORM && active && rt == 0) {
+        // squares of x for the rms scale (the warps of the first row tile see
+        // every chunk once): 4 of the chunk's 128 values per lane
 #pragma unroll
         for (int t = 0; t < NS; ++t) {
           if (t < M) {
@@ -394,15 +404,15 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
     for (int s = 0; s < n_stages; ++s) {
       if (!ptx::mbar_wait(full(slot), phase, err, ptx::wait_code(ptx::kWaitGemvTma, ptx::kWaitFull))) break;
       const uint8_t* st = tsmem + st_off;
-      const int c_first = cb + kSC * s + warp * kCH;
+      const int c_first = cb + kSC * s + wsub * kCHW;
       if (cb + kSC * (s + 1) <= ce) {
         // a whole stage: every chunk is in range
 #pragma unroll
-        for (int h = 0; h < kCH; ++h) chunk(st, warp * kCH + h, c_first + h, true, h == kCH - 1, empty(slot));
+        for (int h = 0; h < kCHW; ++h) chunk(st, wsub * kCHW + h, c_first + h, true, h == kCHW - 1, empty(slot));
       } else {
 #pragma unroll
-        for (int h = 0; h < kCH; ++h)
-          chunk(st, warp * kCH + h, c_first + h, c_first + h < ce, h == kCH - 1, empty(slot));
+        for (int h = 0; h < kCHW; ++h)
+          chunk(st, wsub * kCHW + h, c_first + h, c_first + h < ce, h == kCHW - 1, empty(slot));
       }
       st_off += st_bytes;
       if (++slot == S) {
@@ -427,17 +437,19 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
   }
   __syncthreads();
 
-  // ---- reduce the K slices: warps, then the cluster ----
-  if (warp == 0) {
+  // ---- reduce the K slices: warps, then the cluster; warp t finishes row
+  // tile t ----
+  if (warp < RT) {
+    const int t_row = warp;
     float acc[NT][4];
     float ss[NS];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        float v = red[0][nt][lane][q];
+        float v = red[t_row][nt][lane][q];
 #pragma unroll
-        for (int w2 = 1; w2 < kCW; ++w2) v += red[w2][nt][lane][q];
+        for (int w2 = t_row + RT; w2 < kCW; w2 += RT) v += red[w2][nt][lane][q];
         acc[nt][q] = v;
       }
 #pragma unroll
@@ -451,12 +463,12 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
       ss[t] = v;
     }
     if (KC > 1) {
-      float* dst = cluster.map_shared_rank(&cl_red[0][0][0][0], 0);
+      float* dst = cluster.map_shared_rank(&cl_red[0][0][0][0][0], 0);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) dst[((cr * NT + nt) * 32 + lane) * 4 + q] = acc[nt][q];
-      if (NORM && lane == 0) {
+        for (int q = 0; q < 4; ++q) dst[(((cr * RT + t_row) * NT + nt) * 32 + lane) * 4 + q] = acc[nt][q];
+      if (NORM && t_row == 0 && lane == 0) {
         float* dss = cluster.map_shared_rank(&cl_ss[0][0], 0);
 #pragma unroll
         for (int t = 0; t < NS; ++t) dss[cr * NS + t] = ss[t];
@@ -469,8 +481,8 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            float v = cl_red[0][nt][lane][q];
-            for (int r = 1; r < KC; ++r) v += cl_red[r][nt][lane][q];
+            float v = cl_red[0][t_row][nt][lane][q];
+            for (int r = 1; r < KC; ++r) v += cl_red[r][t_row][nt][lane][q];
             acc[nt][q] = v;
           }
         if (NORM) {
@@ -493,7 +505,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
           inv[e] = 1.0f / sqrtf(v / static_cast<float>(K) + 1e-6f);
         }
       }
-      const int ra = r0 + g, rb = r0 + g + 8;
+      const int ra = r0 + 16 * t_row + g, rb = ra + 8;
       // with group scales the chunks were scaled as they were summed
       const float sca = GRP ? 1.0f : (ra < N ? __ldg(scales + ra) : 0.0f);
       const float scb = GRP ? 1.0f : (rb < N ? __ldg(scales + rb) : 0.0f);
@@ -552,11 +564,14 @@ int cluster_size(int tiles, int chunks, int num_sms) {
 }
 
 // gstride, gshift: group scales (GRP; see the kernel), else unused.
-// MC: as for the kernel (M must then equal MC).
-template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0>
+// MC, RT: as for the kernel (M must equal MC when MC > 0).
+// too_big: if not null, set (and nothing launched) when the configuration's
+// shared memory would not fit one CTA, so that the caller can take fewer row
+// tiles.
+template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0, int RT = 1>
 cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
                     uint16_t* y, bool pdl, int flags, int32_t* err, cudaStream_t stream, int gstride = 0,
-                    int gshift = 0) {
+                    int gshift = 0, bool* too_big = nullptr) {
   auto encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
   const int64_t rb = 16 * ((static_cast<int64_t>(K) * B + 127) / 128);
@@ -570,7 +585,8 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(16 * B), static_cast<cuuint64_t>(N),
                                 static_cast<cuuint64_t>(chunks)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(16 * B)};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(16 * B), 16, static_cast<cuuint32_t>(kSC)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(16 * B), static_cast<cuuint32_t>(16 * RT),
+                               static_cast<cuuint32_t>(kSC)};
     const cuuint32_t estr[3] = {1, 1, 1};
     boxes = encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(packed), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -590,10 +606,10 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
   if (boxes) {
     flags |= kStageBoxes;
   } else {
-    // one 2D TMA per chunk: {16*B bytes x 16 rows} of W, {128 values x M} of x
+    // one 2D TMA per chunk: {16*B bytes x 16*RT rows} of W, {128 values x M} of x
     const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(N)};
     const cuuint64_t wstrides[1] = {static_cast<cuuint64_t>(rb)};
-    const cuuint32_t wbox[2] = {static_cast<cuuint32_t>(16 * B), 16};
+    const cuuint32_t wbox[2] = {static_cast<cuuint32_t>(16 * B), static_cast<cuuint32_t>(16 * RT)};
     const cuuint64_t xdims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
     const cuuint64_t xstrides[1] = {static_cast<cuuint64_t>(K) * 2};
     const cuuint32_t xbox[2] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(M)};
@@ -606,23 +622,33 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC>;
-  const int tiles = (N + 15) / 16;
+  auto kern = gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT>;
+  const int tiles = (N + 16 * RT - 1) / (16 * RT);
   const int kc = cluster_size(tiles, chunks, device_info().num_sms);
   const int per_cta = ((chunks + kc - 1) / kc + kSC - 1) / kSC;
   // resident CTAs per SM that registers and static shared memory allow
   static const int ctas_by_regs = [] {
     int n = 0;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC>, kThreads,
-                                                         0) ==
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT>,
+                                                         kThreads, 0) ==
                    cudaSuccess
                ? n
                : 0;
   }();
-  const uint32_t cl_bytes = kc > 1 ? static_cast<uint32_t>(kc) * NT * 32 * 4 * sizeof(float) : 0u;
+  const uint32_t cl_bytes = kc > 1 ? static_cast<uint32_t>(kc) * RT * NT * 32 * 4 * sizeof(float) : 0u;
   const uint32_t fixed = cl_bytes + static_cast<uint32_t>(sizeof(float)) * kCW * NT * 32 * 4 + 1024u;
-  const int S = ring_stages(B, M, per_cta, tiles * kc <= device_info().num_sms, ctas_by_regs, fixed);
-  const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M) + cl_bytes;
+  const int S = ring_stages(B, M, per_cta, tiles * kc <= device_info().num_sms, ctas_by_regs, fixed, RT);
+  const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M, RT) + cl_bytes;
+  if (too_big != nullptr) {
+    static const size_t static_smem = [] {
+      cudaFuncAttributes a;
+      return cudaFuncGetAttributes(&a, gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT>) == cudaSuccess
+                 ? a.sharedSizeBytes
+                 : size_t{16384};
+    }();
+    *too_big = smem + static_smem > static_cast<size_t>(device_info().max_smem_optin);
+    if (*too_big) return cudaSuccess;
+  }
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
