@@ -59,7 +59,8 @@ def peaks():
 
 # Sources whose change invalidates a committed DRAM-traffic figure for the
 # decode kernel that the headline times.
-TMA_GEMV_SOURCES = ["gemv_tma.cuh", "gemv_tma.cu", "expand.cuh", "tc_ptx.cuh"]
+TMA_GEMV_SOURCES = ["gemv_tma.cuh", "gemv_tma_dispatch.cuh", "gemv_tma.cu", "gemv_tma_canon.cu",
+                    "expand.cuh", "tc_ptx.cuh"]
 
 
 def kernel_source_hash(names):
@@ -412,6 +413,55 @@ def measure_groups(mpw, W_gpu, b, g, l2_bytes, layout, steps, warmup=3):
             "us_per_launch": round(us, 4), "weight_GBps": round(per / (us * 1e3), 1),
             "alg_GBps": round((per + 2 * K + 2 * N) / (us * 1e3), 1),
             "quantize_us": round(q_us, 3), "quantize_GBps": round(q_bytes / (q_us * 1e3), 1)}
+
+
+def measure_sharded(mpw, world, rank, steps=20, warmup=3, layout="paired"):
+    """Output-row sharding across the ranks (every rank calls this; one NCCL
+    all-gather per call): the 27B-class gate matrix 17408x5120, b = 6, split
+    into row blocks, M = 1 and M = 8.  GB/s count the whole matrix's packed
+    bytes over the slowest rank's time per call; the gathered y is checked
+    against the unsharded linear on this rank."""
+    import torch
+    import torch.distributed as dist
+
+    import workloads as wl
+    from mixed_precision_weight_row_b200 import shard
+
+    name, N, K = [s for s in wl.MLP27B["shapes"] if s[0] == "gate"][0]
+    b = 6
+    W = wl.gen_weight_torch(N, K, wl.MLP27B["sigma"], 17 + N)
+    packed, scales = mpw.quantize_pack(W, b)
+    del W
+    if layout != "canonical":
+        packed = mpw.repack(packed, K, b, "canonical", layout)
+    lin = shard.ShardedLinear.from_full(packed, scales, N, K, b, world, rank, layout=layout)
+    out = {"shape": f"{name} {N}x{K}", "b": b, "ranks": world, "rows_per_rank": lin.Nl}
+    for M in (1, 8):
+        x = wl.gen_x(M, K, 1).cuda()
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        for _ in range(warmup):
+            shard.qlinear_sharded(x, lin, y=y)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            shard.qlinear_sharded(x, lin, y=y)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+        full = mpw.qlinear(x, packed, scales, b, layout=layout)
+        torch.cuda.synchronize()
+        diff = float((full.float() - y.float()).abs().max())
+        scale = float(full.float().abs().max())
+        out[f"M{M}"] = {"us_per_call": round(ms * 1e3, 3),
+                        "matrix_GBps": round((packed.numel() + scales.numel() * 4) / (ms * 1e-3) / 1e9, 1),
+                        "max_abs_diff_vs_unsharded": diff, "max_abs_y": scale}
+    del packed, scales, lin
+    torch.cuda.empty_cache()
+    return out
 
 
 def measure_e2e(mpw, packed_host, scales_host, x_host, b, M, N, K, steps, warmup, pool_n, layout="canonical",
@@ -827,8 +877,12 @@ def main(argv=None):
     e2e = sec.run("e2e", measure_e2e, mpw, packed_h, scales_h, x_h, HEADLINE_BITS, 1, N, K,
                   max(3, min(args.steps, 10)), 3, pool.P, layout=lay, world=world)
 
-    # rank 0 alone from here on: no collective until the end
+    # output-row sharding over the ranks (every rank; collectives)
     extras = {}
+    if world > 1:
+        extras["sharded"] = sec.run("sharded", measure_sharded, mpw, world, rank, layout=lay)
+
+    # rank 0 alone from here on: no collective until the end
     if rank == 0:
         # the same launches, each one waiting for its predecessor before it
         # reads x (what a chain of dependent linears sees)
@@ -922,7 +976,7 @@ def main(argv=None):
 
     traffic = profile_traffic(f"gemv_tma_decode_b6_m1_{lay}.json", TMA_GEMV_SOURCES)
     roof = {"bound": "hbm",
-            "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,0,{str(lay == 'paired').lower()},false,1>",
+            "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,0,{str(lay == 'paired').lower()},false,1,1>",
             "achieved": round(achieved, 1) if achieved is not None else None,
             "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / pk["hbm_gbs"], 4) if achieved is not None else None,
