@@ -650,6 +650,16 @@ def measure_recipe(mpw, pk, steps=10, warmup=3, layout="canonical"):
            "tokens_per_s": round(1e3 / per, 2), "weight_GBps": round(wbytes / (per * 1e-3) / 1e9, 1),
            "pct_hbm": round(100 * wbytes / (per * 1e-3) / 1e9 / pk["hbm_gbs"], 2),
            "launches_per_token": len(layers)}
+    if layout == "paired":
+        # the same pass planned as one persistent kernel (mpw_pass_*)
+        p = mpw.Pass(layers, slots, 1)
+        g = graph_of(p.run)
+        ms = time_graph(g, steps, warmup) / steps
+        del g
+        p.close()
+        res["persistent_pass"] = {"ms_per_token": round(ms, 4), "tokens_per_s": round(1e3 / ms, 2),
+                                  "pct_hbm": round(100 * wbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 2),
+                                  "launches_per_token": 1, "note": "opt-in; slower than the per-linear launches"}
     del layers
     torch.cuda.empty_cache()
     return res

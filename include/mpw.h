@@ -69,7 +69,8 @@ typedef enum mpw_status {
   MPW_E_TIMEOUT = 6,          /* a device-side wait gave up (see mpw_device_error) */
   MPW_E_SCRATCH_LIMIT = 7,    /* mpw_qlinear_noalloc: the call needs more than its fixed scratch */
   MPW_E_IO = 8,               /* mpw_file_*: the file cannot be opened, read or written */
-  MPW_E_FORMAT = 9            /* mpw_file_*: not a valid container, truncated, or a checksum differs */
+  MPW_E_FORMAT = 9,           /* mpw_file_*: not a valid container, truncated, or a checksum differs */
+  MPW_E_UNSUPPORTED = 10      /* mpw_pass_create: a linear or M the planned pass does not take */
 } mpw_status;
 
 /* Static English text for a status code; never NULL. */
@@ -344,6 +345,46 @@ MPW_API mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count,
                                      void* workspace, size_t workspace_bytes, mpw_stream_t stream);
 
 /*
+ * mpw_pass_create / mpw_pass_run / mpw_pass_info / mpw_pass_destroy -- the
+ * same decode pass as mpw_recipe_run, planned once and run as ONE persistent
+ * kernel per call.
+ * Pages: DynaQuant "Step 3" (a stack of linears, each at its own bit width)
+ * and "Custom kernel architecture" (in decode the packed bytes streamed are
+ * the cost).  Launched one kernel per linear, a linear that depends on its
+ * predecessor starts on a nearly idle GPU; the planned pass keeps every SM
+ * streaming weights across linears (work items of 16 rows and a run of K;
+ * each linear waits, on the device, only for the earlier linears that write
+ * what it reads or read or write what it writes).
+ *   mpw_pass_create  arguments as mpw_recipe_run (validated alike).  Takes
+ *            M == 1, every linear in MPW_LAYOUT_PAIRED with bits 4..8 and
+ *            K % 128 == 0 (else MPW_E_UNSUPPORTED: use mpw_recipe_run), and
+ *            no linear whose input and output bytes overlap
+ *            (MPW_E_INVALID_ARG).  Allocates device memory for the plan
+ *            (descriptors, TMA tensor maps, dependency lists, counters and
+ *            partial sums: about 128 B per split 16-row tile) and returns it in
+ *            *pass.  The plan records the slot and matrix pointers: they must
+ *            stay valid, and the slots keep their sizes, while it is used.
+ *            Synchronous (host to device copies); not capturable.
+ *   mpw_pass_run  zeroes the plan's counters and launches the kernel on
+ *            `stream` (capturable in a CUDA graph).  One run at a time per
+ *            plan.  Results equal mpw_recipe_run's within the decode
+ *            tolerance (linears split along K add their parts' fp32 sums in a
+ *            fixed order; not bit-identical to the per-linear kernels).
+ *            A device-side wait that gives up sets the error word (kernel 6,
+ *            place 11 for the wait on other linears, see mpw_device_error).
+ *   mpw_pass_info  info[0..3] = grid size (CTAs), ring stages per CTA, work
+ *            items, dynamic shared memory bytes per CTA.
+ *   mpw_pass_destroy  frees the plan (after its last run has completed);
+ *            NULL is a no-op.
+ */
+typedef struct mpw_pass mpw_pass;
+MPW_API mpw_status mpw_pass_create(const mpw_linear* layers, int64_t count, uint16_t* const* slots,
+                                   int64_t num_slots, int64_t M, mpw_pass** pass);
+MPW_API mpw_status mpw_pass_run(const mpw_pass* pass, mpw_stream_t stream);
+MPW_API mpw_status mpw_pass_info(const mpw_pass* pass, int64_t* info);
+MPW_API void mpw_pass_destroy(mpw_pass* pass);
+
+/*
  * mpw_allocate_bits -- per-matrix bit widths under a byte budget.
  * Pages: DynaQuant "Step 2: bit allocation" (water filling over a max-heap of
  * marginal bit upgrades: each step raises one matrix to its next level, by
@@ -518,13 +559,17 @@ MPW_API mpw_status mpw_gather_shards(const uint16_t* blocks, int64_t world, int6
  *   other  the first bounded wait (2 s of waiting) inside a TMA / tensor-core
  *          kernel that gave up, as 100 * kernel + place: kernel 1 = per-tile
  *          decode, 2 = tensor-memory decode, 3 = prefill GEMM, 4 = stream-K
- *          decode, 5 = FP8 prefill GEMM; place 1 = x producer waiting for a free stage, 2 = x
+ *          decode, 5 = FP8 prefill GEMM, 6 = planned decode pass (mpw_pass_run);
+ *          place 1 = x producer waiting for a free stage, 2 = x
  *          producer waiting for its last copies, 3 / 4 = the same for the
  *          weight (or combined) producer, 5 = consumer or MMA issuer waiting
  *          for a loaded stage, 6 = MMA issuer waiting for converted weights,
  *          7 = converter waiting for a loaded weight stage, 8 = converter
  *          waiting for a free tensor-memory stage, 9 = epilogue waiting for
- *          the accumulator, 10 = sums of squares waiting for a loaded x stage.
+ *          the accumulator, 10 = sums of squares waiting for a loaded x stage,
+ *          11 = a pass item waiting for the linears it depends on.  In the
+ *          planned pass the other waits give up soon after the first one
+ *          did (without codes of their own).
  *          The outputs of the call that gave up, and of calls that depend
  *          on them, are undefined.
  */

@@ -18,7 +18,7 @@ from dataclasses import dataclass
 __all__ = [
     "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
     "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str", "allocate_bits", "allocation_frontier",
-    "recipe_plan", "save_packed", "load_packed",
+    "recipe_plan", "save_packed", "load_packed", "Pass",
     "LAYOUTS", "workspace", "qlinear_workspace_bytes", "quantize_pack_groups", "qlinear_groups",
     "gather_shards", "quantize_x_fp8", "qlinear_fp8",
 ]
@@ -35,6 +35,7 @@ MPW_E_TIMEOUT = 6
 MPW_E_SCRATCH_LIMIT = 7
 MPW_E_IO = 8
 MPW_E_FORMAT = 9
+MPW_E_UNSUPPORTED = 10
 
 PATHS = {"auto": 0, "gemv": 1, "gemm": 2}
 # Packed layouts (mpw_layout): the canonical stream and its paired-halves
@@ -136,6 +137,14 @@ def _load():
     L.mpw_qlinear_noalloc.restype = c_int
     L.mpw_recipe_run.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, vp]
     L.mpw_recipe_run.restype = c_int
+    L.mpw_pass_create.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64, ctypes.POINTER(vp)]
+    L.mpw_pass_create.restype = c_int
+    L.mpw_pass_run.argtypes = [vp, vp]
+    L.mpw_pass_run.restype = c_int
+    L.mpw_pass_info.argtypes = [vp, ctypes.POINTER(i64)]
+    L.mpw_pass_info.restype = c_int
+    L.mpw_pass_destroy.argtypes = [vp]
+    L.mpw_pass_destroy.restype = None
     L.mpw_quantize_pack_groups.argtypes = [vp, i64, i64, c_int, i64, vp, vp, vp, vp]
     L.mpw_quantize_pack_groups.restype = c_int
     L.mpw_qlinear_groups.argtypes = [vp, vp, vp, c_int, i64, c_int, i64, i64, i64, vp, ctypes.c_uint, vp]
@@ -566,6 +575,52 @@ def recipe_plan(layers, slots, M: int):
     flags = (ctypes.c_uint32 * len(layers))()
     _check(lib.mpw_recipe_plan(arr, len(layers), ptrs, len(slots), int(M), flags), "mpw_recipe_plan")
     return list(flags)
+
+
+def _linear_array(layers):
+    arr = (_Linear * len(layers))()
+    for i, L in enumerate(layers):
+        arr[i] = _Linear(L.packed.data_ptr(), L.scales.data_ptr(), int(L.N), int(L.K), int(L.bits),
+                         int(L.in_slot), int(L.out_slot), int(bool(L.norm_input)), LAYOUTS[L.layout], 0)
+    return arr
+
+
+class Pass:
+    """A decode pass planned once and run as one persistent kernel per call
+    (mpw_pass_create / mpw_pass_run).  Holds references to the layers' and
+    slots' tensors, whose pointers the plan records.  Raises MPWError with
+    MPW_E_UNSUPPORTED when the pass does not take these linears."""
+
+    def __init__(self, layers, slots, M: int = 1):
+        arr = _linear_array(layers)
+        ptrs = (ctypes.c_void_p * len(slots))(*[s.data_ptr() for s in slots])
+        h = ctypes.c_void_p()
+        _check(lib.mpw_pass_create(arr, len(layers), ptrs, len(slots), int(M), ctypes.byref(h)), "mpw_pass_create")
+        self._h = h
+        self._keep = (list(layers), list(slots))
+
+    def run(self, stream=None) -> None:
+        if not self._h:
+            raise ValueError("pass already closed")
+        _check(lib.mpw_pass_run(self._h, _stream(stream)), "mpw_pass_run")
+
+    def info(self) -> dict:
+        v = (ctypes.c_int64 * 4)()
+        _check(lib.mpw_pass_info(self._h, v), "mpw_pass_info")
+        return {"grid": v[0], "stages": v[1], "items": v[2], "smem_bytes": v[3]}
+
+    def close(self) -> None:
+        """Free the plan (the caller makes sure its last run has completed)."""
+        if self._h:
+            lib.mpw_pass_destroy(self._h)
+            self._h = ctypes.c_void_p()
+            self._keep = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def recipe_run(layers, slots, M: int, stream=None, use_workspace: bool = False):

@@ -126,6 +126,7 @@ const char* mpw_status_str(int status) {
     case MPW_E_SCRATCH_LIMIT: return "call needs more than the fixed scratch of mpw_qlinear_noalloc";
     case MPW_E_IO: return "file cannot be opened, read or written";
     case MPW_E_FORMAT: return "not a valid packed-weight file, or a checksum differs";
+    case MPW_E_UNSUPPORTED: return "the planned decode pass does not take these linears (use mpw_recipe_run)";
     default: return "unknown status";
   }
 }
@@ -425,6 +426,52 @@ mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count, uint16_t* con
                           int64_t num_slots, int64_t M, mpw_stream_t stream) {
   return mpw_recipe_run_ws(layers, count, slots, num_slots, M, nullptr, 0, stream);
 }
+
+mpw_status mpw_pass_create(const mpw_linear* layers, int64_t count, uint16_t* const* slots, int64_t num_slots,
+                           int64_t M, mpw_pass** pass) {
+  if (pass == nullptr) return MPW_E_INVALID_ARG;
+  *pass = nullptr;
+  const mpw_status st = recipe_check(layers, count, slots, num_slots, M);
+  if (st != MPW_OK) return st;
+  if (M != 1 || count > (1 << 20)) return MPW_E_UNSUPPORTED;
+  std::vector<mpw::PassLayer> pl(static_cast<size_t>(count));
+  for (int64_t i = 0; i < count; ++i) {
+    const mpw_linear& L = layers[i];
+    if (!mpw::gemv_pass_layer_ok(L.bits, L.layout, L.N, L.K)) return MPW_E_UNSUPPORTED;
+    mpw::PassLayer& P = pl[static_cast<size_t>(i)];
+    P.x = slots[L.in_slot];
+    P.y = slots[L.out_slot];
+    P.packed = L.packed;
+    P.scales = L.scales;
+    P.N = L.N;
+    P.K = L.K;
+    P.bits = L.bits;
+    P.norm = L.norm_input != 0;
+    // a linear whose input and output bytes overlap cannot be ordered
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(P.x), ya = reinterpret_cast<uintptr_t>(P.y);
+    if (xa < ya + 2u * static_cast<uintptr_t>(P.N) && ya < xa + 2u * static_cast<uintptr_t>(P.K))
+      return MPW_E_INVALID_ARG;
+  }
+  mpw::PassPlan* plan = nullptr;
+  const cudaError_t e = mpw::gemv_pass_create(pl.data(), count, &plan);
+  if (e != cudaSuccess) return MPW_E_CUDA;
+  *pass = reinterpret_cast<mpw_pass*>(plan);
+  return MPW_OK;
+}
+
+mpw_status mpw_pass_run(const mpw_pass* pass, mpw_stream_t stream) {
+  if (pass == nullptr) return MPW_E_INVALID_ARG;
+  return from_cuda(mpw::gemv_pass_run(reinterpret_cast<const mpw::PassPlan*>(pass),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+mpw_status mpw_pass_info(const mpw_pass* pass, int64_t* info) {
+  if (pass == nullptr || info == nullptr) return MPW_E_INVALID_ARG;
+  mpw::gemv_pass_info(reinterpret_cast<const mpw::PassPlan*>(pass), info);
+  return MPW_OK;
+}
+
+void mpw_pass_destroy(mpw_pass* pass) { mpw::gemv_pass_destroy(reinterpret_cast<mpw::PassPlan*>(pass)); }
 
 mpw_status mpw_device_error(int32_t* code) {
   if (code == nullptr) return MPW_E_INVALID_ARG;

@@ -155,4 +155,25 @@ cudaError_t launch_gemm(const uint16_t* x, const uint8_t* packed, const float* s
                         int32_t* dev_error, cudaStream_t stream);
 bool gemm_supported(int64_t M, int64_t N, int64_t K);
 
+// gemv_pass.cu: a decode pass (one token) over a stack of linears as one
+// persistent kernel.  A plan owns its device memory (descriptors, tensor maps,
+// dependency lists, counters, partial sums); the pointers in the layers must
+// stay valid while it is used.
+struct PassLayer {
+  const uint16_t* x;       // input, K values
+  uint16_t* y;             // output, N values
+  const uint8_t* packed;   // paired rows
+  const float* scales;
+  int64_t N, K;
+  int bits;
+  bool norm;
+};
+struct PassPlan;
+bool gemv_pass_layer_ok(int bits, int layout, int64_t N, int64_t K);
+cudaError_t gemv_pass_create(const PassLayer* layers, int64_t count, PassPlan** out);
+cudaError_t gemv_pass_run(const PassPlan* plan, cudaStream_t stream);
+void gemv_pass_destroy(PassPlan* plan);
+// grid size, ring stages, work items, dynamic shared memory bytes
+void gemv_pass_info(const PassPlan* plan, int64_t* info);
+
 }  // namespace mpw

@@ -66,7 +66,9 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 
 // Codes a wait that gives up leaves in the device error word:
 // 100 * kernel + place.  The first one stays until the word is read.
-enum WaitKernel : int32_t { kWaitGemvTma = 1, kWaitGemvTc = 2, kWaitGemm = 3, kWaitGemvSk = 4, kWaitGemmFp8 = 5 };
+enum WaitKernel : int32_t {
+  kWaitGemvTma = 1, kWaitGemvTc = 2, kWaitGemm = 3, kWaitGemvSk = 4, kWaitGemmFp8 = 5, kWaitGemvPass = 6
+};
 enum WaitPlace : int32_t {
   kWaitXEmpty = 1,    // x producer: a free x stage
   kWaitXTail = 2,     // x producer: its last copies landed
@@ -78,6 +80,7 @@ enum WaitPlace : int32_t {
   kWaitAEmpty = 8,    // converter: a free tensor-memory stage
   kWaitAcc = 9,       // epilogue: the finished accumulator
   kWaitSquares = 10,  // sums of squares of x: a loaded x stage
+  kWaitDeps = 11,     // decode pass: the linears this one depends on, finished
 };
 __host__ __device__ constexpr int32_t wait_code(int32_t kernel, int32_t place) { return 100 * kernel + place; }
 
@@ -107,6 +110,79 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int32_t
     prev = now;
     if (waited > limit_ns || round >= kWaitMaxRounds) {
       if (err != nullptr) atomicCAS(err, 0, code);
+      return false;
+    }
+  }
+}
+
+// mbar_wait for kernels whose CTAs wait on one another: a wait that gives up
+// also sets *abort (a word of the launch's own, zero at its start), and every
+// wait gives up (without a code of its own) soon after *abort is set, so that
+// one failed wait does not leave every other CTA waiting out its full limit.
+__device__ __forceinline__ bool mbar_wait_abortable(uint32_t bar, uint32_t parity, int32_t* err, int32_t code,
+                                                    int32_t* abort, uint64_t limit_ns = 2000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t prev = globaltimer();
+  uint64_t waited = 0;
+#pragma unroll 1
+  for (uint32_t round = 0;; ++round) {
+#pragma unroll 1
+    for (int i = 0; i < 128; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t now = globaltimer();
+    if (now > prev) waited += (now - prev < kWaitMaxStepNs) ? now - prev : kWaitMaxStepNs;
+    prev = now;
+    if ((round & 63u) == 63u && *reinterpret_cast<volatile int32_t*>(abort) != 0) return false;
+    if (waited > limit_ns || round >= kWaitMaxRounds) {
+      atomicCAS(err, 0, code);
+      atomicExch(abort, 1);
+      return false;
+    }
+  }
+}
+
+// ---- counters in global memory (gpu scope) ------------------------------------
+
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(int32_t* p, int32_t v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int32_t atom_add_acq_rel_gpu(int32_t* p, int32_t v) {
+  int32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Orders this thread's generic-proxy accesses of global memory with its later
+// async-proxy (TMA, bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Waits until *counter >= target (acquire): bounded like mbar_wait_abortable.
+__device__ __forceinline__ bool counter_wait(const int32_t* counter, int32_t target, int32_t* err, int32_t code,
+                                             int32_t* abort, uint64_t limit_ns = 2000000000ull) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  uint64_t prev = globaltimer();
+  uint64_t waited = 0;
+#pragma unroll 1
+  for (uint32_t round = 0;; ++round) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (ld_acquire_gpu(counter) >= target) return true;
+    const uint64_t now = globaltimer();
+    if (now > prev) waited += (now - prev < kWaitMaxStepNs) ? now - prev : kWaitMaxStepNs;
+    prev = now;
+    if ((round & 63u) == 63u && *reinterpret_cast<volatile int32_t*>(abort) != 0) return false;
+    if (waited > limit_ns || round >= kWaitMaxRounds) {
+      atomicCAS(err, 0, code);
+      atomicExch(abort, 1);
       return false;
     }
   }
@@ -145,6 +221,22 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
       : "memory");
+}
+
+// Untiled bulk copy global -> shared (both 16-byte aligned, bytes a multiple
+// of 16), completing `bytes` transactions on the mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Prefetch of a tiled box into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int32_t c0, int32_t c1, int32_t c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
