@@ -378,6 +378,17 @@ MPW_API mpw_status mpw_recipe_run_ws(const mpw_linear* layers, int64_t count,
  *            NULL is a no-op.
  */
 typedef struct mpw_pass mpw_pass;
+/* mpw_pass_dependencies -- host only: the earlier linears each linear of the
+ * planned pass waits for (those that write bytes it reads, or read or write
+ * bytes it writes, minus those another listed one waits for, transitively):
+ * linear i waits for deps[offsets[i] .. offsets[i+1]).  offsets has count + 1
+ * entries and is always filled on success of the validation; deps must hold
+ * offsets[count] entries (else MPW_E_INVALID_ARG, with offsets filled).
+ * Arguments and errors as mpw_pass_create; slot pointers are compared, never
+ * dereferenced. */
+MPW_API mpw_status mpw_pass_dependencies(const mpw_linear* layers, int64_t count, uint16_t* const* slots,
+                                         int64_t num_slots, int64_t M, int32_t* offsets, int32_t* deps,
+                                         int64_t deps_capacity);
 MPW_API mpw_status mpw_pass_create(const mpw_linear* layers, int64_t count, uint16_t* const* slots,
                                    int64_t num_slots, int64_t M, mpw_pass** pass);
 MPW_API mpw_status mpw_pass_run(const mpw_pass* pass, mpw_stream_t stream);

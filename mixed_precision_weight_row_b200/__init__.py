@@ -18,7 +18,7 @@ from dataclasses import dataclass
 __all__ = [
     "MPWError", "LIB_PATH", "lib", "packed_row_bytes", "quantize_pack", "unpack",
     "dequantize", "repack", "qlinear", "Linear", "recipe_run", "device_error", "status_str", "allocate_bits", "allocation_frontier",
-    "recipe_plan", "save_packed", "load_packed", "Pass",
+    "recipe_plan", "save_packed", "load_packed", "Pass", "pass_dependencies",
     "LAYOUTS", "workspace", "qlinear_workspace_bytes", "quantize_pack_groups", "qlinear_groups",
     "gather_shards", "quantize_x_fp8", "qlinear_fp8",
 ]
@@ -145,6 +145,9 @@ def _load():
     L.mpw_pass_info.restype = c_int
     L.mpw_pass_destroy.argtypes = [vp]
     L.mpw_pass_destroy.restype = None
+    L.mpw_pass_dependencies.argtypes = [ctypes.POINTER(_Linear), i64, ctypes.POINTER(vp), i64, i64,
+                                        ctypes.POINTER(i32), ctypes.POINTER(i32), i64]
+    L.mpw_pass_dependencies.restype = c_int
     L.mpw_quantize_pack_groups.argtypes = [vp, i64, i64, c_int, i64, vp, vp, vp, vp]
     L.mpw_quantize_pack_groups.restype = c_int
     L.mpw_qlinear_groups.argtypes = [vp, vp, vp, c_int, i64, c_int, i64, i64, i64, vp, ctypes.c_uint, vp]
@@ -577,12 +580,34 @@ def recipe_plan(layers, slots, M: int):
     return list(flags)
 
 
+def _addr(t) -> int:
+    return t if isinstance(t, int) else t.data_ptr()
+
+
 def _linear_array(layers):
     arr = (_Linear * len(layers))()
     for i, L in enumerate(layers):
-        arr[i] = _Linear(L.packed.data_ptr(), L.scales.data_ptr(), int(L.N), int(L.K), int(L.bits),
+        arr[i] = _Linear(_addr(L.packed), _addr(L.scales), int(L.N), int(L.K), int(L.bits),
                          int(L.in_slot), int(L.out_slot), int(bool(L.norm_input)), LAYOUTS[L.layout], 0)
     return arr
+
+
+def pass_dependencies(layers, slots, M: int = 1):
+    """For every linear, the earlier linears the planned pass makes it wait
+    for (mpw_pass_dependencies; host only, slot addresses are compared, never
+    read).  ``slots`` may be tensors or plain integer addresses."""
+    arr = _linear_array(layers)
+    addr = [s if isinstance(s, int) else s.data_ptr() for s in slots]
+    ptrs = (ctypes.c_void_p * len(slots))(*addr)
+    offsets = (ctypes.c_int32 * (len(layers) + 1))()
+    st = lib.mpw_pass_dependencies(arr, len(layers), ptrs, len(slots), int(M), offsets, None, 0)
+    need = offsets[len(layers)]
+    if st != MPW_OK and not (st == MPW_E_INVALID_ARG and need > 0):
+        _check(st, "mpw_pass_dependencies")
+    deps = (ctypes.c_int32 * max(need, 1))()
+    _check(lib.mpw_pass_dependencies(arr, len(layers), ptrs, len(slots), int(M), offsets, deps, need),
+           "mpw_pass_dependencies")
+    return [list(deps[offsets[i]:offsets[i + 1]]) for i in range(len(layers))]
 
 
 class Pass:

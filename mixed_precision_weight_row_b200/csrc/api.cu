@@ -427,14 +427,13 @@ mpw_status mpw_recipe_run(const mpw_linear* layers, int64_t count, uint16_t* con
   return mpw_recipe_run_ws(layers, count, slots, num_slots, M, nullptr, 0, stream);
 }
 
-mpw_status mpw_pass_create(const mpw_linear* layers, int64_t count, uint16_t* const* slots, int64_t num_slots,
-                           int64_t M, mpw_pass** pass) {
-  if (pass == nullptr) return MPW_E_INVALID_ARG;
-  *pass = nullptr;
+// The planned pass's view of a recipe: one PassLayer per linear (host only).
+mpw_status pass_layers(const mpw_linear* layers, int64_t count, uint16_t* const* slots, int64_t num_slots,
+                       int64_t M, std::vector<mpw::PassLayer>& pl) {
   const mpw_status st = recipe_check(layers, count, slots, num_slots, M);
   if (st != MPW_OK) return st;
   if (M != 1 || count > (1 << 20)) return MPW_E_UNSUPPORTED;
-  std::vector<mpw::PassLayer> pl(static_cast<size_t>(count));
+  pl.assign(static_cast<size_t>(count), mpw::PassLayer{});
   for (int64_t i = 0; i < count; ++i) {
     const mpw_linear& L = layers[i];
     if (!mpw::gemv_pass_layer_ok(L.bits, L.layout, L.N, L.K)) return MPW_E_UNSUPPORTED;
@@ -452,6 +451,31 @@ mpw_status mpw_pass_create(const mpw_linear* layers, int64_t count, uint16_t* co
     if (xa < ya + 2u * static_cast<uintptr_t>(P.N) && ya < xa + 2u * static_cast<uintptr_t>(P.K))
       return MPW_E_INVALID_ARG;
   }
+  return MPW_OK;
+}
+
+mpw_status mpw_pass_dependencies(const mpw_linear* layers, int64_t count, uint16_t* const* slots,
+                                 int64_t num_slots, int64_t M, int32_t* offsets, int32_t* deps,
+                                 int64_t deps_capacity) {
+  if (offsets == nullptr || deps_capacity < 0 || (deps == nullptr && deps_capacity > 0)) return MPW_E_INVALID_ARG;
+  std::vector<mpw::PassLayer> pl;
+  const mpw_status st = pass_layers(layers, count, slots, num_slots, M, pl);
+  if (st != MPW_OK) return st;
+  std::vector<int32_t> d, d0;
+  if (!mpw::gemv_pass_dependencies(pl.data(), count, d, d0)) return MPW_E_INVALID_ARG;
+  for (int64_t i = 0; i <= count; ++i) offsets[i] = d0[static_cast<size_t>(i)];
+  if (static_cast<int64_t>(d.size()) > deps_capacity) return MPW_E_INVALID_ARG;
+  for (size_t i = 0; i < d.size(); ++i) deps[i] = d[i];
+  return MPW_OK;
+}
+
+mpw_status mpw_pass_create(const mpw_linear* layers, int64_t count, uint16_t* const* slots, int64_t num_slots,
+                           int64_t M, mpw_pass** pass) {
+  if (pass == nullptr) return MPW_E_INVALID_ARG;
+  *pass = nullptr;
+  std::vector<mpw::PassLayer> pl;
+  const mpw_status st = pass_layers(layers, count, slots, num_slots, M, pl);
+  if (st != MPW_OK) return st;
   mpw::PassPlan* plan = nullptr;
   const cudaError_t e = mpw::gemv_pass_create(pl.data(), count, &plan);
   if (e != cudaSuccess) return MPW_E_CUDA;

@@ -494,6 +494,38 @@ struct PassPlan {
   size_t smem = 0;
 };
 
+bool gemv_pass_dependencies(const PassLayer* layers, int64_t count, std::vector<int32_t>& deps,
+                            std::vector<int32_t>& dep0) {
+  // conflicting earlier linears, minus those another listed one already
+  // covers (ancestor sets as bitsets; scanned from the nearest linear back)
+  const int L = static_cast<int>(count);
+  const int words = (L + 63) / 64;
+  std::vector<uint64_t> anc(static_cast<size_t>(L) * words, 0ull);
+  deps.clear();
+  dep0.assign(static_cast<size_t>(L) + 1, 0);
+  for (int i = 0; i < L; ++i) {
+    const PassLayer& A = layers[i];
+    const Range in{reinterpret_cast<uintptr_t>(A.x), reinterpret_cast<uintptr_t>(A.x) + 2u * A.K};
+    const Range outr{reinterpret_cast<uintptr_t>(A.y), reinterpret_cast<uintptr_t>(A.y) + 2u * A.N};
+    if (in.overlaps(outr)) return false;
+    uint64_t* mine = anc.data() + static_cast<size_t>(i) * words;
+    dep0[static_cast<size_t>(i)] = static_cast<int32_t>(deps.size());
+    for (int jx = i - 1; jx >= 0; --jx) {
+      if (mine[jx / 64] >> (jx % 64) & 1ull) continue;   // covered already
+      const PassLayer& Bj = layers[jx];
+      const Range bin{reinterpret_cast<uintptr_t>(Bj.x), reinterpret_cast<uintptr_t>(Bj.x) + 2u * Bj.K};
+      const Range bout{reinterpret_cast<uintptr_t>(Bj.y), reinterpret_cast<uintptr_t>(Bj.y) + 2u * Bj.N};
+      if (!(bout.overlaps(in) || bin.overlaps(outr) || bout.overlaps(outr))) continue;
+      deps.push_back(jx);
+      const uint64_t* theirs = anc.data() + static_cast<size_t>(jx) * words;
+      for (int w = 0; w < words; ++w) mine[w] |= theirs[w];
+      mine[jx / 64] |= 1ull << (jx % 64);
+    }
+  }
+  dep0[static_cast<size_t>(L)] = static_cast<int32_t>(deps.size());
+  return true;
+}
+
 bool gemv_pass_layer_ok(int bits, int layout, int64_t N, int64_t K) {
   return layout == kLayoutPaired && bits >= 4 && bits <= 8 && K >= 128 && K % 128 == 0 && N >= 1 &&
          N < (1LL << 30) && K < (1LL << 30);
@@ -524,32 +556,13 @@ cudaError_t gemv_pass_create(const PassLayer* layers, int64_t count, PassPlan** 
   if (occ < 1) return cudaErrorInvalidConfiguration;
   const long long G = static_cast<long long>(occ) * d.num_sms;
 
-  // dependencies: conflicting earlier linears, minus those another listed one
-  // already covers (ancestor sets as bitsets)
-  const int words = (L + 63) / 64;
-  std::vector<uint64_t> anc(static_cast<size_t>(L) * words, 0ull);
-  std::vector<int32_t> deps;
+  std::vector<int32_t> deps, dep0;
+  if (!gemv_pass_dependencies(layers, count, deps, dep0)) return cudaErrorInvalidValue;
   std::vector<PassLinear> lin(static_cast<size_t>(L));
   long long items = 0, recs = 0;
   int cnts = 0;
   for (int i = 0; i < L; ++i) {
     const PassLayer& A = layers[i];
-    const Range in{reinterpret_cast<uintptr_t>(A.x), reinterpret_cast<uintptr_t>(A.x) + 2u * A.K};
-    const Range outr{reinterpret_cast<uintptr_t>(A.y), reinterpret_cast<uintptr_t>(A.y) + 2u * A.N};
-    if (in.overlaps(outr)) return cudaErrorInvalidValue;
-    uint64_t* mine = anc.data() + static_cast<size_t>(i) * words;
-    const int dep0 = static_cast<int>(deps.size());
-    for (int jx = i - 1; jx >= 0; --jx) {
-      if (mine[jx / 64] >> (jx % 64) & 1ull) continue;   // covered already
-      const PassLayer& Bj = layers[jx];
-      const Range bin{reinterpret_cast<uintptr_t>(Bj.x), reinterpret_cast<uintptr_t>(Bj.x) + 2u * Bj.K};
-      const Range bout{reinterpret_cast<uintptr_t>(Bj.y), reinterpret_cast<uintptr_t>(Bj.y) + 2u * Bj.N};
-      if (!(bout.overlaps(in) || bin.overlaps(outr) || bout.overlaps(outr))) continue;
-      deps.push_back(jx);
-      const uint64_t* theirs = anc.data() + static_cast<size_t>(jx) * words;
-      for (int w = 0; w < words; ++w) mine[w] |= theirs[w];
-      mine[jx / 64] |= 1ull << (jx % 64);
-    }
     PassLinear& P = lin[static_cast<size_t>(i)];
     P.x = A.x;
     P.y = A.y;
@@ -565,8 +578,8 @@ cudaError_t gemv_pass_create(const PassLayer* layers, int64_t count, PassPlan** 
     long long parts = G / P.tiles;
     parts = std::min<long long>(std::max<long long>(parts, 1), P.stages);
     P.parts = static_cast<int>(parts);
-    P.dep0 = dep0;
-    P.ndep = static_cast<int>(deps.size()) - dep0;
+    P.dep0 = dep0[static_cast<size_t>(i)];
+    P.ndep = dep0[static_cast<size_t>(i) + 1] - dep0[static_cast<size_t>(i)];
     P.item0 = items;
     items += static_cast<long long>(P.tiles) * P.parts;
     P.rec0 = recs;

@@ -9,6 +9,8 @@
 #include <stdint.h>
 #include <stdlib.h>
 
+#include <vector>
+
 namespace mpw {
 
 constexpr int kMinBits = 4;
@@ -170,6 +172,10 @@ struct PassLayer {
 };
 struct PassPlan;
 bool gemv_pass_layer_ok(int bits, int layout, int64_t N, int64_t K);
+// Host only: for every linear the earlier linears it waits for (deps
+// [dep0[i], dep0[i+1])); false if a linear's input and output overlap.
+bool gemv_pass_dependencies(const PassLayer* layers, int64_t count, std::vector<int32_t>& deps,
+                            std::vector<int32_t>& dep0);
 cudaError_t gemv_pass_create(const PassLayer* layers, int64_t count, PassPlan** out);
 cudaError_t gemv_pass_run(const PassPlan* plan, cudaStream_t stream);
 void gemv_pass_destroy(PassPlan* plan);
