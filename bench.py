@@ -986,7 +986,7 @@ def main(argv=None):
 
     traffic = profile_traffic(f"gemv_tma_decode_b6_m1_{lay}.json", TMA_GEMV_SOURCES)
     roof = {"bound": "hbm",
-            "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,0,{str(lay == 'paired').lower()},false,1,1>",
+            "kernel": f"gemv_tma_kernel<{HEADLINE_BITS},1,0,{str(lay == 'paired').lower()},false,1,1,8>",
             "achieved": round(achieved, 1) if achieved is not None else None,
             "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / pk["hbm_gbs"], 4) if achieved is not None else None,

@@ -470,11 +470,16 @@ cudaError_t launch_gemv(const uint16_t* x, const uint8_t* packed, const float* s
     const char* e = tuning_env("MPW_GEMV_KERNEL");
     return e != nullptr && e[0] == 't' && e[1] == 'c';
   }();
+  // MPW_GEMV_KERNEL=tma: never the tensor-memory kernel (tuning aid)
+  static const bool no_tc = [] {
+    const char* e = tuning_env("MPW_GEMV_KERNEL");
+    return e != nullptr && e[0] == 't' && e[1] == 'm';
+  }();
   // Tensor-memory kernel (passes of 32 tokens) where it is the faster one
   // (MPW_GEMV_KERNEL=tc forces it, a tuning aid).
   {
     const int64_t m1 = M < 32 ? M : 32;
-    if (ws == nullptr && !use_mma && gemv_tc_supported(x, m1, N, K, norm_input) &&
+    if (ws == nullptr && !use_mma && !no_tc && gemv_tc_supported(x, m1, N, K, norm_input) &&
         (use_tc || gemv_tc_preferred(bits, m1, N, K))) {
       for (int64_t m0 = 0; m0 < M; m0 += 32) {
         const int64_t mt = M - m0 < 32 ? M - m0 : 32;

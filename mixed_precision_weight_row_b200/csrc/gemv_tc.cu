@@ -448,11 +448,13 @@ cudaError_t tc_bits(const uint16_t* x, int M, const uint8_t* packed, const float
 
 template <int B>
 bool tc_preferred(int64_t M, int64_t N, int64_t K) {
-  // measured: this kernel wins over the per-tile decode kernel from M = 16
-  // (M = 9 for b >= 8) when each CTA streams a long K slice; with a short
-  // slice its fixed costs (tensor-memory set-up, pipeline fill, cluster
+  // measured: this kernel wins over the per-tile decode kernel (two row
+  // tiles, four-chunk stages) above 16 tokens when each CTA streams a long K
+  // slice (gate 17408x5120 / down 5120x17408, b = 6, M = 32: 29 / 21%
+  // against 20 / 19% of HBM), not at 16 (30 / 24% against 37 / 35%); with a
+  // short slice its fixed costs (tensor-memory set-up, pipeline fill, cluster
   // gather) dominate
-  if (M <= 8 || (B <= 7 && M < 16)) return false;
+  if (M <= 16) return false;
   const int tiles = static_cast<int>((N + BM - 1) / BM);
   const int wbs = static_cast<int>((K + WB - 1) / WB);
   const int kc = tc_cluster<B>(tiles, wbs, static_cast<int>(M < BN ? M : BN), device_info().num_sms);

@@ -10,14 +10,14 @@
 //
 // A CTA owns a 16-row tile of W (a cluster of 1..8 CTAs splits the tile's K
 // range).  The last warp is the producer: one lane fills a ring of stages of
-// kCW*kCH 128-code chunks each (mbarrier completion).  When K % 128 == 0 a
+// SC (8, or 4) 128-code chunks each (mbarrier completion).  When K % 128 == 0 a
 // stage is two 3D TMAs: the packed rows viewed as [chunk][row][16*B bytes]
-// ({16*B x 16 rows x 8 chunks}) and x viewed as [chunk][token][128 values]
-// ({128 x M x 8 chunks}); rows past N and chunks past K read as zeros.  One
+// ({16*B x 16 rows x SC chunks}) and x viewed as [chunk][token][128 values]
+// ({128 x M x SC chunks}); rows past N and chunks past K read as zeros.  One
 // thread issuing many small copies is slow (tens of nanoseconds each), so
 // large boxes matter.  Other K take one 2D TMA per chunk and operand (bytes
 // past the row and values past K read as zeros).  Shared memory holds the
-// same [chunk][row] and [chunk][token] layout either way.  Consumer warp w takes kCH consecutive
+// same [chunk][row] and [chunk][token] layout either way.  Consumer warp w takes SC / 4 consecutive
 // chunks of each stage: per chunk, the 32-code group of lane tig for rows g
 // and g+8 (B words per row) and its x fragment for token g, both from shared
 // memory; it expands the codes to exact bf16 (expand.cuh; canonical or
@@ -75,10 +75,10 @@ constexpr int kXReady = 1;              // flags: x is not written by the preced
 constexpr int kStageBoxes = 2;          // flags: one 3D TMA per stage and operand
 constexpr int kYFree = 4;               // flags: no call of the run touches y
 
-// Bytes of one stage: kSC weight chunks (16*RT rows x 16*B bytes) followed
-// by kSC x chunks (M tokens x 128 bf16).
-__host__ __device__ constexpr uint32_t stage_bytes(int B, int M, int RT = 1) {
-  return static_cast<uint32_t>(kSC) * 256u * static_cast<uint32_t>(B * RT + M);
+// Bytes of one stage: SC weight chunks (16*RT rows x 16*B bytes) followed
+// by SC x chunks (M tokens x 128 bf16).
+__host__ __device__ constexpr uint32_t stage_bytes(int B, int M, int RT = 1, int SC = kSC) {
+  return static_cast<uint32_t>(SC) * 256u * static_cast<uint32_t>(B * RT + M);
 }
 
 // Ring depth.  When the grid fits on the SMs in one wave, a CTA whose whole
@@ -91,13 +91,14 @@ __host__ __device__ constexpr uint32_t stage_bytes(int B, int M, int RT = 1) {
 // MPW_GEMV_RING_KB replaces the rule by a fixed budget (tuning aid).
 constexpr uint32_t kWholeSlice = 64u * 1024u;
 
-int ring_stages(int B, int M, int stages_per_cta, bool few_ctas, int ctas_by_regs, uint32_t fixed, int RT = 1) {
+int ring_stages(int B, int M, int stages_per_cta, bool few_ctas, int ctas_by_regs, uint32_t fixed, int RT = 1,
+                int SC = kSC) {
   static const uint32_t budget = [] {
     const char* e = tuning_env("MPW_GEMV_RING_KB");
     const int v = e ? atoi(e) : 0;
     return v >= 8 && v <= 192 ? static_cast<uint32_t>(v) * 1024u : 0u;
   }();
-  const uint32_t st = stage_bytes(B, M, RT);
+  const uint32_t st = stage_bytes(B, M, RT, SC);
   int s;
   if (budget != 0) {
     s = static_cast<int>(budget / st);
@@ -169,8 +170,10 @@ constexpr int min_ctas_for() {
 // RT: 16-row tiles per CTA.  The RT tiles share each stage's x chunks (x is
 // loaded once for 16*RT rows instead of once per 16), which matters when
 // several tokens make x as large as the weights; consumer warp w takes tile
-// w % RT and 2*RT of the stage's chunks.
-template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0, int RT = 1>
+// w % RT and (SC / 4) * RT of the stage's chunks.
+// SC: 128-code chunks per stage (8, or 4 when x makes stages so large that
+// shared memory would hold too few CTAs).
+template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0, int RT = 1, int SC = kSC>
 __global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, NSQ, PAIRED>())
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                 int M_, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
@@ -181,11 +184,12 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
   constexpr bool NORM = NSQ > 0;
   constexpr int NS = NSQ > 0 ? NSQ : 1;
   static_assert(RT == 1 || RT == 2 || RT == 4, "row tiles per CTA");
+  static_assert(SC == 4 || SC == 8, "chunks per stage");
   constexpr uint32_t kWChunk = 256u * B * RT;   // 16*RT rows x 16*B bytes
-  constexpr int kCHW = kCH * RT;                // chunks per consumer warp and stage
+  constexpr int kCHW = (SC / kCW) * RT;         // chunks per consumer warp and stage
   const uint32_t x_chunk = 256u * M;            // M tokens x 128 bf16
-  const uint32_t w_part = kSC * kWChunk;
-  const uint32_t st_bytes = stage_bytes(B, M, RT);
+  const uint32_t w_part = SC * kWChunk;
+  const uint32_t st_bytes = stage_bytes(B, M, RT, SC);
   // dynamic: the ring (S stages), then, in clusters, the partial sums of the
   // cluster's CTAs
   extern __shared__ __align__(128) uint8_t tsmem[];
@@ -195,7 +199,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
   __shared__ float cl_ss[8][NS];
   __shared__ __align__(16) uint4 zero_x[4];   // x fragment of lanes without a token
   // cluster partial sums: [cluster rank][row tile][NT][32][4]
-  auto cl_red = reinterpret_cast<float (*)[RT][NT][32][4]>(tsmem + static_cast<uint32_t>(S) * stage_bytes(B, M, RT));
+  auto cl_red = reinterpret_cast<float (*)[RT][NT][32][4]>(tsmem + static_cast<uint32_t>(S) * stage_bytes(B, M, RT, SC));
 
   if (flags & kXReady) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cg::cluster_group cluster = cg::this_cluster();
@@ -208,7 +212,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
   const int cpc = (chunks + KC - 1) / KC;
   const int cb = cr * cpc;
   const int ce = min(chunks, cb + cpc);
-  const int n_stages = ce > cb ? (ce - cb + kSC - 1) / kSC : 0;
+  const int n_stages = ce > cb ? (ce - cb + SC - 1) / SC : 0;
   const int r0 = tile * 16 * RT;
   const uint32_t base = ptx::smem_addr(tsmem);
   const uint32_t bar0 = ptx::smem_addr(bars);
@@ -231,9 +235,9 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
       ptx::prefetch_tmap(&tmap_w);
       ptx::prefetch_tmap(&tmap_x);
       const bool boxes = (flags & kStageBoxes) != 0;
-      auto nvalid = [&](int s) { return min(kSC, ce - (cb + kSC * s)); };
+      auto nvalid = [&](int s) { return min(SC, ce - (cb + SC * s)); };
       auto issue_w = [&](int s, int slot) {
-        const int c0 = cb + kSC * s, nv = nvalid(s);
+        const int c0 = cb + SC * s, nv = nvalid(s);
         if (boxes) {
           // a box lands whole (zeros past the tensor); chunks past this
           // CTA's range are loaded and not read
@@ -246,7 +250,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
           ptx::tma_load_2d(base + slot * st_bytes + j * kWChunk, &tmap_w, full(slot), (c0 + j) * 16 * B, r0);
       };
       auto issue_x = [&](int s, int slot) {
-        const int c0 = cb + kSC * s, nv = nvalid(s);
+        const int c0 = cb + SC * s, nv = nvalid(s);
         if (boxes) {
           ptx::tma_load_3d(base + slot * st_bytes + w_part, &tmap_x, full(slot), 0, 0, c0);
           return;
@@ -404,8 +408,8 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
     for (int s = 0; s < n_stages; ++s) {
       if (!ptx::mbar_wait(full(slot), phase, err, ptx::wait_code(ptx::kWaitGemvTma, ptx::kWaitFull))) break;
       const uint8_t* st = tsmem + st_off;
-      const int c_first = cb + kSC * s + wsub * kCHW;
-      if (cb + kSC * (s + 1) <= ce) {
+      const int c_first = cb + SC * s + wsub * kCHW;
+      if (cb + SC * (s + 1) <= ce) {
         // a whole stage: every chunk is in range
 #pragma unroll
         for (int h = 0; h < kCHW; ++h) chunk(st, wsub * kCHW + h, c_first + h, true, h == kCHW - 1, empty(slot));
@@ -564,11 +568,11 @@ int cluster_size(int tiles, int chunks, int num_sms) {
 }
 
 // gstride, gshift: group scales (GRP; see the kernel), else unused.
-// MC, RT: as for the kernel (M must equal MC when MC > 0).
+// MC, RT, SC: as for the kernel (M must equal MC when MC > 0).
 // too_big: if not null, set (and nothing launched) when the configuration's
 // shared memory would not fit one CTA, so that the caller can take fewer row
 // tiles.
-template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0, int RT = 1>
+template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0, int RT = 1, int SC = kSC>
 cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
                     uint16_t* y, bool pdl, int flags, int32_t* err, cudaStream_t stream, int gstride = 0,
                     int gshift = 0, bool* too_big = nullptr) {
@@ -586,7 +590,7 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
                                 static_cast<cuuint64_t>(chunks)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(rb), static_cast<cuuint64_t>(16 * B)};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(16 * B), static_cast<cuuint32_t>(16 * RT),
-                               static_cast<cuuint32_t>(kSC)};
+                               static_cast<cuuint32_t>(SC)};
     const cuuint32_t estr[3] = {1, 1, 1};
     boxes = encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(packed), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -597,7 +601,7 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
                                 static_cast<cuuint64_t>(chunks)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * 2, static_cast<cuuint64_t>(kChunk) * 2};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(kChunk), static_cast<cuuint32_t>(M),
-                               static_cast<cuuint32_t>(kSC)};
+                               static_cast<cuuint32_t>(SC)};
     const cuuint32_t estr[3] = {1, 1, 1};
     boxes = encode(&tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -622,14 +626,14 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kern = gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT>;
+  auto kern = gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT, SC>;
   const int tiles = (N + 16 * RT - 1) / (16 * RT);
   const int kc = cluster_size(tiles, chunks, device_info().num_sms);
-  const int per_cta = ((chunks + kc - 1) / kc + kSC - 1) / kSC;
+  const int per_cta = ((chunks + kc - 1) / kc + SC - 1) / SC;
   // resident CTAs per SM that registers and static shared memory allow
   static const int ctas_by_regs = [] {
     int n = 0;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT>,
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT, SC>,
                                                          kThreads, 0) ==
                    cudaSuccess
                ? n
@@ -637,12 +641,12 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
   }();
   const uint32_t cl_bytes = kc > 1 ? static_cast<uint32_t>(kc) * RT * NT * 32 * 4 * sizeof(float) : 0u;
   const uint32_t fixed = cl_bytes + static_cast<uint32_t>(sizeof(float)) * kCW * NT * 32 * 4 + 1024u;
-  const int S = ring_stages(B, M, per_cta, tiles * kc <= device_info().num_sms, ctas_by_regs, fixed, RT);
-  const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M, RT) + cl_bytes;
+  const int S = ring_stages(B, M, per_cta, tiles * kc <= device_info().num_sms, ctas_by_regs, fixed, RT, SC);
+  const size_t smem = static_cast<size_t>(S) * stage_bytes(B, M, RT, SC) + cl_bytes;
   if (too_big != nullptr) {
     static const size_t static_smem = [] {
       cudaFuncAttributes a;
-      return cudaFuncGetAttributes(&a, gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT>) == cudaSuccess
+      return cudaFuncGetAttributes(&a, gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT, SC>) == cudaSuccess
                  ? a.sharedSizeBytes
                  : size_t{16384};
     }();

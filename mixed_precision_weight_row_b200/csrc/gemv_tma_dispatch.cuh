@@ -21,28 +21,56 @@ inline int row_tiles_for(int M) {
   if (forced > 0) return forced;
   // measured on 4096x4096 (b = 4, 6) and the 27B-class gate/down matrices:
   // two tiles win from M = 4 to 32 (e.g. M = 8, b = 6: 48 -> 55% of HBM),
-  // four lose (too few CTAs per SM to hide latency)
+  // four lose (too few CTAs per SM to hide latency; built in tuning builds
+  // only)
   return M == 1 ? 1 : 2;
+}
+
+// 128-code chunks per ring stage for a pass of M tokens: eight, or four when
+// the x chunks make stages so large that shared memory holds few CTAs
+// (MPW_GEMV_SC sets it in a tuning build).
+inline int stage_chunks_for(int M) {
+  static const int forced = [] {
+    const char* e = tuning_env("MPW_GEMV_SC");
+    const int v = e ? atoi(e) : 0;
+    return (v == 4 || v == 8) ? v : 0;
+  }();
+  if (forced > 0) return forced;
+  // measured (two row tiles): four chunks from M = 4 (4096x4096 b = 6: M = 4
+  // / 8 / 16 from 78 / 55 / 28 to 87 / 67 / 38% of HBM; gate 17408x5120 M = 8
+  // from 59 to 66%, down 5120x17408 from 52 to 60%), where stages of eight
+  // chunks leave shared memory for only two CTAs per SM
+  return M >= 4 ? 4 : 8;
+}
+
+template <int B, bool PAIRED, int NT, int SC>
+cudaError_t tma_rt_sc(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
+                      uint16_t* y, bool pdl, int flags, int32_t* err, cudaStream_t stream) {
+  // fewer row tiles when a ring of two stages would not fit one CTA's shared
+  // memory (wide codes with many tokens)
+  const int rt = row_tiles_for(M);
+  bool too_big = false;
+#ifdef MPW_TUNING_KNOBS
+  if (rt == 4) {
+    const cudaError_t e = run_tma<B, NT, 0, PAIRED, false, 0, 4, SC>(x, M, packed, scales, N, K, y, pdl, flags,
+                                                                      err, stream, 0, 0, &too_big);
+    if (e != cudaSuccess || !too_big) return e;
+  }
+#endif
+  if (rt >= 2) {
+    const cudaError_t e = run_tma<B, NT, 0, PAIRED, false, 0, 2, SC>(x, M, packed, scales, N, K, y, pdl, flags,
+                                                                      err, stream, 0, 0, &too_big);
+    if (e != cudaSuccess || !too_big) return e;
+  }
+  return run_tma<B, NT, 0, PAIRED, false, 0, 1, SC>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
 }
 
 template <int B, bool PAIRED, int NT>
 cudaError_t tma_rt(const uint16_t* x, int M, const uint8_t* packed, const float* scales, int N, int K,
                    uint16_t* y, bool pdl, int flags, int32_t* err, cudaStream_t stream) {
-  // fewer row tiles when a ring of two stages would not fit one CTA's shared
-  // memory (wide codes with many tokens)
-  const int rt = row_tiles_for(M);
-  bool too_big = false;
-  if (rt == 4) {
-    const cudaError_t e = run_tma<B, NT, 0, PAIRED, false, 0, 4>(x, M, packed, scales, N, K, y, pdl, flags, err,
-                                                                  stream, 0, 0, &too_big);
-    if (e != cudaSuccess || !too_big) return e;
-  }
-  if (rt >= 2) {
-    const cudaError_t e = run_tma<B, NT, 0, PAIRED, false, 0, 2>(x, M, packed, scales, N, K, y, pdl, flags, err,
-                                                                  stream, 0, 0, &too_big);
-    if (e != cudaSuccess || !too_big) return e;
-  }
-  return run_tma<B, NT, 0, PAIRED>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  if (stage_chunks_for(M) == 4)
+    return tma_rt_sc<B, PAIRED, NT, 4>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
+  return tma_rt_sc<B, PAIRED, NT, 8>(x, M, packed, scales, N, K, y, pdl, flags, err, stream);
 }
 
 template <int B, bool PAIRED>

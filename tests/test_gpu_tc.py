@@ -1,6 +1,6 @@
 """The tensor-memory decode kernel (weights expanded into tensor memory,
-tcgen05 MMAs with a 32-token tile), which the decode path selects for M > 8
-on shapes with long K slices.  Sampled rows are compared with the oracle
+tcgen05 MMAs with a 32-token tile), which the decode path selects for M > 16
+on shapes with long K slices (M = 16 is also run: the per-tile kernel then).  Sampled rows are compared with the oracle
 (each output row depends on one weight row only); the whole kernel was also
 run over the full decode parity suite with it forced (MPW_GEMV_KERNEL=tc).
 """
@@ -52,11 +52,11 @@ def test_tc_decode_sampled_rows(mpw, weights, b, layout, M):
 def test_tc_one_hot_exact(mpw):
     import torch
 
-    b, M = 8, 16
+    b, M = 8, 17
     rng = np.random.default_rng(5)
     q = rng.integers(-127, 128, size=(N, K)).astype(np.int32)
     s = (rng.random(N).astype(np.float32) + np.float32(0.5)) * np.float32(0.01)
-    ks = np.array([0, 1, 127, 128, 1000, 2047, 2048, 3071, 5, 6, 7, 8, 9, 10, 11, 12])
+    ks = np.array([0, 1, 127, 128, 1000, 2047, 2048, 3071, 5, 6, 7, 8, 9, 10, 11, 12, 3000])
     x = torch.zeros((M, K), dtype=torch.bfloat16)
     for m, k in enumerate(ks):
         x[m, k] = 1.0
