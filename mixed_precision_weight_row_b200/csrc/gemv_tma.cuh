@@ -542,13 +542,19 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constan
 // host side
 // ---------------------------------------------------------------------------
 
-// Cluster size: each 16-row tile is one cluster of kc CTAs.  Time is modelled
-// as (CTAs per SM) x (chunks per consumer warp + a fixed cost of three chunks
-// for start-up and the reduction).
-int cluster_size(int tiles, int chunks, int num_sms) {
+// Cluster size: each tile is one cluster of kc CTAs.  One token: time is
+// modelled as (CTAs per SM) x (chunks per consumer warp + a fixed cost of
+// three chunks for start-up and the reduction), which splits K where the
+// tiles alone leave SMs idle (down 5120x17408: two CTAs per tile; a recipe
+// pass of dependent launches is 9% faster for it).  Several tokens: one CTA
+// per tile (measured on gate 17408x5120 and down 5120x17408 at M = 4, 8, 16
+// with two-tile CTAs: every split was slower, down M = 8 b = 6 60 against 66%
+// of HBM).  The choice depends on the shape and M only, never on the call's
+// flags, so that flagged and unflagged calls give the same bits.
+int cluster_size(int tiles, int chunks, int num_sms, int M) {
   int best = 1;
   double best_t = 1e300;
-  for (int kc = 1; kc <= 8; kc *= 2) {
+  for (int kc = 1; kc <= (M == 1 ? 8 : 1); kc *= 2) {
     if (kc > 1 && kCW * kc > chunks) break;
     const double per_sm = std::ceil(static_cast<double>(tiles) * kc / num_sms);
     const double cpw = std::ceil(static_cast<double>(chunks) / (kCW * kc));
@@ -628,7 +634,7 @@ cudaError_t run_tma(const uint16_t* x, int M, const uint8_t* packed, const float
   }
   auto kern = gemv_tma_kernel<B, NT, NSQ, PAIRED, GRP, MC, RT, SC>;
   const int tiles = (N + 16 * RT - 1) / (16 * RT);
-  const int kc = cluster_size(tiles, chunks, device_info().num_sms);
+  const int kc = cluster_size(tiles, chunks, device_info().num_sms, M);
   const int per_cta = ((chunks + kc - 1) / kc + SC - 1) / SC;
   // resident CTAs per SM that registers and static shared memory allow
   static const int ctas_by_regs = [] {
