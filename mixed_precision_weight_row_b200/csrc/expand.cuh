@@ -196,6 +196,13 @@ __device__ __forceinline__ uint32_t paired_field(const uint32_t (&w)[B + 1]) {
   uint32_t t;
   if constexpr (r + NB <= 16) {
     t = r == 0 ? w[h] : (w[h] >> r);
+  } else if constexpr (r >= 8 && r + NB <= 24) {
+    // the field lies in the top byte of each half of word h and the bottom
+    // byte of each half of word h+1: one byte permute gathers both halves'
+    // 16-bit windows (even stream low, odd stream high), then one shift
+    uint32_t u;
+    asm("prmt.b32 %0, %1, %2, 0x6341;" : "=r"(u) : "r"(w[h]), "r"(w[h + 1]));
+    t = u >> (r - 8);
   } else {
     // low part from word h, high part from word h+1, in both halves at once
     constexpr uint32_t sel = ((1u << (16 - r)) - 1u) * 0x10001u;
