@@ -150,13 +150,14 @@ constexpr int dec_parts() {
   return PAIRED ? GemmParts<B>::parts : Exp<B>::parts;
 }
 
-// Paired rows with one part and one token tile fit in 64 registers (56 for
-// b <= 5): six or seven CTAs per SM; the rms-scaled variant for one token
-// needs a few more (five CTAs), the one for up to eight tokens keeps eight
-// sums of squares and stays at four.
+// Paired rows with one part and one token tile fit in 56 registers up to
+// b = 7 (seven CTAs per SM, no spills) and 64 at b = 8, 9 (six); the
+// rms-scaled variant for one token needs a few more (five CTAs), the one for
+// up to eight tokens keeps eight sums of squares and stays at four.
 template <int B, int NT, int NSQ, bool PAIRED>
 constexpr int min_ctas_for() {
-  return PAIRED && dec_parts<B, PAIRED>() == 1 && NT == 1 ? (NSQ > 1 ? 4 : (NSQ == 1 ? 5 : 6)) : min_ctas<B, NT>();
+  return PAIRED && dec_parts<B, PAIRED>() == 1 && NT == 1 ? (NSQ > 1 ? 4 : (NSQ == 1 ? 5 : (B <= 7 ? 7 : 6)))
+                                                          : min_ctas<B, NT>();
 }
 
 // NSQ: 0 = plain input; 1 or kNormMaxM = rms-scaled input for up to that
