@@ -151,13 +151,15 @@ constexpr int dec_parts() {
 }
 
 // Paired rows with one part and one token tile fit in 56 registers up to
-// b = 7 (seven CTAs per SM, no spills) and 64 at b = 8, 9 (six); the
+// b = 7 (seven CTAs per SM, no spills) and 64 at b = 8, 9 (six); with group
+// scales (GRP) they need up to 64 (six; at 56 they would spill); the
 // rms-scaled variant for one token needs a few more (five CTAs), the one for
 // up to eight tokens keeps eight sums of squares and stays at four.
-template <int B, int NT, int NSQ, bool PAIRED>
+template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false>
 constexpr int min_ctas_for() {
-  return PAIRED && dec_parts<B, PAIRED>() == 1 && NT == 1 ? (NSQ > 1 ? 4 : (NSQ == 1 ? 5 : (B <= 7 ? 7 : 6)))
-                                                          : min_ctas<B, NT>();
+  return PAIRED && dec_parts<B, PAIRED>() == 1 && NT == 1
+             ? (NSQ > 1 ? 4 : (NSQ == 1 ? 5 : (B <= 7 && !GRP ? 7 : 6)))
+             : min_ctas<B, NT>();
 }
 
 // NSQ: 0 = plain input; 1 or kNormMaxM = rms-scaled input for up to that
@@ -175,7 +177,7 @@ constexpr int min_ctas_for() {
 // SC: 128-code chunks per stage (8, or 4 when x makes stages so large that
 // shared memory would hold too few CTAs).
 template <int B, int NT, int NSQ, bool PAIRED, bool GRP = false, int MC = 0, int RT = 1, int SC = kSC>
-__global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, NSQ, PAIRED>())
+__global__ void __launch_bounds__(kThreads, min_ctas_for<B, NT, NSQ, PAIRED, GRP>())
 gemv_tma_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                 int M_, const float* __restrict__ scales, int N, int K, uint16_t* __restrict__ y, int S,
                 int flags, int32_t* err, int gstride, int gshift) {
