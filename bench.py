@@ -746,7 +746,7 @@ def run_case(args):
         _, N, K = wl.PREFILL["shapes"][0]
         W = wl.gen_weight_torch(N, K, wl.PREFILL["sigma"], 11 + N)
         M = wl.PREFILL["M"]
-    if args.case == "recipe":
+    if args.case in ("recipe", "pass"):
         shapes, bits, links = wl.recipe_shapes(1), wl.recipe_bits()[:7], wl.recipe_links(1)
         layers = []
         for i, ((_, _, N, K), bb, (si, so, nrm)) in enumerate(zip(shapes, bits, links)):
@@ -755,8 +755,16 @@ def run_case(args):
                 mpw.repack(packed, K, bb, "canonical", args.layout, out=packed)
             layers.append(mpw.Linear(packed, scales, N, K, bb, si, so, nrm, layout=args.layout))
         slots = [torch.zeros((1, wl.SLOT_WIDTH[s]), dtype=torch.bfloat16, device="cuda") for s in range(8)]
-        for _ in range(args.launches):
-            mpw.recipe_run(layers, slots, 1)
+        if args.case == "pass":
+            # one layer of the recipe stack as one persistent kernel
+            p = mpw.Pass(layers, slots, 1)
+            for _ in range(args.launches):
+                p.run()
+            torch.cuda.synchronize()
+            p.close()
+        else:
+            for _ in range(args.launches):
+                mpw.recipe_run(layers, slots, 1)
     elif args.case == "quantize":
         for _ in range(args.launches):
             mpw.quantize_pack(W, b)
@@ -809,7 +817,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
-    ap.add_argument("--case", choices=["decode", "gate", "down", "prefill", "recipe", "quantize", "groups",
+    ap.add_argument("--case", choices=["decode", "gate", "down", "prefill", "recipe", "pass", "quantize", "groups",
                                        "prefill_fp8"],
                     default=None, help="profiling target: run a few launches of one kernel, print nothing")
     ap.add_argument("--bits", type=int, default=HEADLINE_BITS, help="bit width for --case")
